@@ -1,0 +1,236 @@
+"""ctypes binding of libint8lt.so (include/int8lt.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+torch supplies device memory and streams. There is no CPU fallback: if the
+shared library is missing or the device is not a B200 (sm_100a), calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libint8lt.so")
+
+STATUS = {
+    0: "INT8LT_OK", 1: "INT8LT_ERR_NULL", 2: "INT8LT_ERR_SHAPE", 3: "INT8LT_ERR_ALIGN",
+    4: "INT8LT_ERR_VALUE", 5: "INT8LT_ERR_WORKSPACE", 6: "INT8LT_ERR_CUDA",
+    7: "INT8LT_ERR_TIMEOUT", 8: "INT8LT_ERR_UNSUPPORTED",
+}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+# Every symbol include/int8lt.h declares.
+EXPORTS = [
+    "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
+    "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
+    "int8lt_forward", "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
+]
+
+
+class Int8ltError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg}")
+        self.status = status
+        self.name = STATUS.get(status, "UNKNOWN")
+
+
+_lock = threading.Lock()
+_lib = None
+
+_P, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_SIGS = {
+    "int8lt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "int8lt_version": (ctypes.c_int, []),
+    "int8lt_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "int8lt_workspace_init": (ctypes.c_int, [_P, _SZ, _P]),
+    "int8lt_read_device_status": (ctypes.c_int, [_P, _SZ, _P]),
+    "int8lt_prepare_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "int8lt_quantize_rows": (ctypes.c_int, [_P, _I64, _I64, _F, _P, _P, _P, _P, _P, _SZ, _P]),
+    "int8lt_forward": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P, _SZ, _P]),
+    "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
+}
+
+
+def lib(path: str | None = None) -> ctypes.CDLL:
+    """Load libint8lt.so (in-tree build); raises if it has not been built."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m bit_quantized_matmul_int8_b200.build`")
+            _lib = _bind(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _bind(l: ctypes.CDLL) -> ctypes.CDLL:
+    for name, (res, args) in _SIGS.items():
+        f = getattr(l, name)
+        f.restype = res
+        f.argtypes = args
+    return l
+
+
+def _check(fn: str, st: int) -> None:
+    if st != 0:
+        raise Int8ltError(fn, st, lib().int8lt_status_string(st).decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------ entry points --
+
+def int8lt_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib().int8lt_workspace_size(M, N, K))
+
+
+def int8lt_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check("int8lt_workspace_init",
+           lib().int8lt_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def int8lt_read_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Status code (0 = OK, 7 = a kernel timed out); clears the status word."""
+    return int(lib().int8lt_read_device_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def workspace(M: int, N: int, K: int, device=None) -> torch.Tensor:
+    """Allocate (uint8) and initialise a workspace for an [M,K] x [N,K]^T call."""
+    n = int8lt_workspace_size(M, N, K)
+    if n == 0:
+        raise Int8ltError("int8lt_workspace_size", 2, f"unsupported shape M={M} N={N} K={K}")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    int8lt_workspace_init(ws)
+    return ws
+
+
+def int8lt_prepare_weight(W: torch.Tensor, CB: torch.Tensor | None = None,
+                          SCB: torch.Tensor | None = None, stream=None):
+    """W fp16 [N,K] -> (CB int8 [N,K], SCB fp32 [N])."""
+    _dev(W, torch.float16, "W")
+    N, K = W.shape
+    CB = torch.empty((N, K), dtype=torch.int8, device=W.device) if CB is None else CB
+    SCB = torch.empty(N, dtype=torch.float32, device=W.device) if SCB is None else SCB
+    _check("int8lt_prepare_weight",
+           lib().int8lt_prepare_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
+    return CB, SCB
+
+
+def int8lt_quantize_rows(X: torch.Tensor, threshold: float = 6.0, ws: torch.Tensor | None = None,
+                         stream=None):
+    """X fp16 [M,K] -> (CA int8 [M,K], SCA fp32 [M], outlier_idx int32 [|O|])."""
+    _dev(X, torch.float16, "X")
+    M, K = X.shape
+    dev = X.device
+    CA = torch.empty((M, K), dtype=torch.int8, device=dev)
+    SCA = torch.empty(M, dtype=torch.float32, device=dev)
+    idx = torch.empty(max(K, 1), dtype=torch.int32, device=dev)
+    n = torch.zeros(1, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(M, 8, K, dev)
+    _check("int8lt_quantize_rows",
+           lib().int8lt_quantize_rows(_ptr(X), M, K, float(threshold), _ptr(CA), _ptr(SCA),
+                                      _ptr(idx), _ptr(n), _ptr(ws), ws.numel(), _stream(stream)))
+    return CA, SCA, idx[: int(n.item())]
+
+
+def int8lt_forward(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                   W_outlier: torch.Tensor | None, threshold: float = 6.0,
+                   bias: torch.Tensor | None = None, Y: torch.Tensor | None = None,
+                   ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y fp16 [M,N] = LLM.int8() forward of X fp16 [M,K] with CB/SCB (and fp16 outlier weights)."""
+    _dev(X, torch.float16, "X")
+    _dev(CB, torch.int8, "CB")
+    _dev(SCB, torch.float32, "SCB")
+    if W_outlier is not None:
+        _dev(W_outlier, torch.float16, "W_outlier")
+    if bias is not None:
+        _dev(bias, torch.float16, "bias")
+    M, K = X.shape
+    N = CB.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(M, N, K, X.device)
+    _check("int8lt_forward",
+           lib().int8lt_forward(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier),
+                                float(threshold), _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(),
+                                _stream(stream)))
+    return Y
+
+
+def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, ws: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    _dev(CA, torch.int8, "CA")
+    _dev(CB, torch.int8, "CB")
+    M, K = CA.shape
+    N = CB.shape[0]
+    C = torch.empty((M, N), dtype=torch.int32, device=CA.device)
+    if ws is None:
+        ws = workspace(M, N, K, CA.device)
+    _check("int8lt_debug_gemm_i32",
+           lib().int8lt_debug_gemm_i32(_ptr(CA), _ptr(CB), M, N, K, _ptr(C), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+    return C
+
+
+def int8lt_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    _check("int8lt_debug_wait_timeout",
+           lib().int8lt_debug_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
+
+
+class Int8Linear:
+    """LLM.int8() linear layer: Y = X W^T + bias with outlier decomposition.
+
+    The counterpart of the Hugging Face ``Linear8bitLt(..., has_fp16_weights=False,
+    threshold=6.0)``: the fp16 weight is converted once (``int8lt_prepare_weight``) and
+    the forward runs ``int8lt_forward``. ``keep_fp16_outlier_weights=False`` drops the
+    fp16 weight and takes the outlier columns' weights from CB * SCB / 127.
+    """
+
+    def __init__(self, weight: torch.Tensor, bias: torch.Tensor | None = None,
+                 threshold: float = 6.0, keep_fp16_outlier_weights: bool = True):
+        self.N, self.K = weight.shape
+        self.threshold = float(threshold)
+        self.CB, self.SCB = int8lt_prepare_weight(weight.contiguous())
+        self.W_outlier = weight.contiguous() if keep_fp16_outlier_weights else None
+        self.bias = bias
+        self._ws: dict[int, torch.Tensor] = {}
+
+    def workspace_for(self, M: int, device) -> torch.Tensor:
+        ws = self._ws.get(M)
+        if ws is None:
+            ws = self._ws[M] = workspace(M, self.N, self.K, device)
+        return ws
+
+    def __call__(self, X: torch.Tensor, Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        ws = self.workspace_for(X.shape[0], X.device)
+        return int8lt_forward(X, self.CB, self.SCB, self.W_outlier, self.threshold, self.bias,
+                              Y, ws, stream)

@@ -1,0 +1,282 @@
+// C ABI of libint8lt: argument validation, workspace layout and dispatch.
+// Every check runs on the host before the first launch; see include/int8lt.h
+// for the contract of each entry point.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+
+#include "int8lt_internal.cuh"
+
+namespace int8lt {
+
+int64_t flag_chunks_for(int64_t M, int64_t K) {
+    const int64_t gx = ceil_div(K, kColsPerFlagCta);
+    int64_t c = ceil_div(2 * 148, gx);
+    c = std::min<int64_t>(c, kMaxFlagChunks);
+    c = std::min<int64_t>(c, ceil_div(std::max<int64_t>(M, 1), 32));
+    return std::max<int64_t>(c, 1);
+}
+
+static size_t align_up(size_t v) { return (v + 1023) & ~size_t(1023); }
+
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
+    WsLayout L{};
+    L.M = M; L.N = N; L.K = K;
+    L.kwords = ceil_div(K, 32);
+    L.kcap = round_up(K, 64);
+    L.flag_chunks = flag_chunks_for(M, K);
+    size_t off = 0;
+    L.hdr = off;   off += align_up(sizeof(WsHeader));
+    L.flags = off; off += align_up((size_t)L.flag_chunks * L.kwords * 4);
+    L.idx = off;   off += align_up((size_t)K * 4);
+    L.sca = off;   off += align_up((size_t)M * 4);
+    L.ca = off;    off += align_up((size_t)M * K);
+    L.xo = off;    off += align_up((size_t)M * L.kcap * 2);
+    if (M > kDecodeMaxM) {
+        L.wo = off; off += align_up((size_t)N * L.kcap * 2);
+        L.acc = L.cnt = SIZE_MAX;
+    } else {
+        L.wo = SIZE_MAX;
+        L.acc = off; off += align_up((size_t)N * 16 * 4);
+        L.cnt = off; off += align_up((size_t)ceil_div(N, 32) * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+}  // namespace int8lt
+
+using namespace int8lt;
+
+namespace {
+
+template <typename T>
+T *at(void *ws, size_t off) {
+    return off == SIZE_MAX ? nullptr : reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool shape_ok(int64_t M, int64_t N, int64_t K) {
+    return M >= 0 && N >= 0 && K >= 16 && K <= kMaxK && (K % 16) == 0 && (N % 8) == 0 &&
+           M <= (int64_t)1 << 31 && N <= (int64_t)1 << 31;
+}
+
+// 0 = unknown, 1 = compute capability 10.0, 2 = other
+std::atomic<int> g_dev_ok[64];
+
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return INT8LT_ERR_CUDA;
+    std::atomic<int> &slot = g_dev_ok[dev & 63];
+    int st = slot.load(std::memory_order_relaxed);
+    if (st == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return INT8LT_ERR_CUDA;
+        st = (major == 10 && minor == 0) ? 1 : 2;
+        slot.store(st, std::memory_order_relaxed);
+    }
+    return st == 1 ? INT8LT_OK : INT8LT_ERR_UNSUPPORTED;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? INT8LT_OK : INT8LT_ERR_CUDA; }
+
+__global__ void wait_timeout_kernel(uint32_t *status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_barrier_init();
+        // Nothing ever arrives on `bar`: the bounded wait must give up.
+        if (!mbar_wait_bounded(smem_u32(&bar), 0, limit_ns)) record_timeout(status);
+    }
+}
+
+}  // namespace
+
+namespace int8lt {
+cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_t s) {
+    wait_timeout_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+}  // namespace int8lt
+
+extern "C" {
+
+const char *int8lt_status_string(int status) {
+    switch (status) {
+        case INT8LT_OK: return "INT8LT_OK";
+        case INT8LT_ERR_NULL: return "INT8LT_ERR_NULL: a required pointer is NULL";
+        case INT8LT_ERR_SHAPE: return "INT8LT_ERR_SHAPE: M, N or K outside the supported limits";
+        case INT8LT_ERR_ALIGN: return "INT8LT_ERR_ALIGN: a pointer is not aligned as required";
+        case INT8LT_ERR_VALUE: return "INT8LT_ERR_VALUE: threshold is NaN or negative";
+        case INT8LT_ERR_WORKSPACE: return "INT8LT_ERR_WORKSPACE: workspace too small";
+        case INT8LT_ERR_CUDA: return "INT8LT_ERR_CUDA: a CUDA call or launch failed";
+        case INT8LT_ERR_TIMEOUT: return "INT8LT_ERR_TIMEOUT: a kernel gave up a bounded wait";
+        case INT8LT_ERR_UNSUPPORTED: return "INT8LT_ERR_UNSUPPORTED: device is not compute capability 10.0";
+        default: return "INT8LT_ERR_UNKNOWN";
+    }
+}
+
+int int8lt_version(void) { return 100; }
+
+size_t int8lt_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (!shape_ok(M, N, K)) return 0;
+    return ws_layout(M, N, K).total;
+}
+
+int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws) return INT8LT_ERR_NULL;
+    if (ws_bytes < sizeof(WsHeader)) return INT8LT_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return INT8LT_ERR_ALIGN;
+    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+}
+
+int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws) return INT8LT_ERR_NULL;
+    if (ws_bytes < sizeof(WsHeader)) return INT8LT_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t status = 0;
+    if (cudaMemcpyAsync(&status, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return INT8LT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return INT8LT_ERR_CUDA;
+    if (status == 0) return INT8LT_OK;
+    if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        return INT8LT_ERR_CUDA;
+    return (status & kStatusTimeout) ? INT8LT_ERR_TIMEOUT : INT8LT_ERR_CUDA;
+}
+
+int int8lt_prepare_weight(const void *W, int64_t N, int64_t K, int8_t *CB, float *SCB, void *stream) {
+    if (!W || !CB || !SCB) return INT8LT_ERR_NULL;
+    if (N < 0 || K < 1 || K > ((int64_t)1 << 31)) return INT8LT_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(CB, 16) || !aligned(SCB, 4)) return INT8LT_ERR_ALIGN;
+    if (N == 0) return INT8LT_OK;
+    if (int st = check_device()) return st;
+    return from_cuda(launch_prepare_weight(static_cast<const __half *>(W), N, K, CB, SCB,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold, int8_t *CA, float *SCA,
+                         int32_t *outlier_idx, int32_t *n_outliers, void *ws, size_t ws_bytes, void *stream) {
+    if (!X || !CA || !SCA || !outlier_idx || !n_outliers || !ws) return INT8LT_ERR_NULL;
+    if (!shape_ok(M, 8, K)) return INT8LT_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(CA, 16) || !aligned(SCA, 4) || !aligned(outlier_idx, 4) ||
+        !aligned(n_outliers, 4) || !aligned(ws, 16))
+        return INT8LT_ERR_ALIGN;
+    if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
+    const WsLayout L = ws_layout(M, 8, K);
+    if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
+    if (M == 0) {
+        // |O| of an empty batch is 0.
+        if (int st = check_device()) return st;
+        return from_cuda(cudaMemsetAsync(n_outliers, 0, 4, static_cast<cudaStream_t>(stream)));
+    }
+    if (int st = check_device()) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t tb = threshold_bits(threshold);
+    uint32_t *flags = at<uint32_t>(ws, L.flags);
+    if (cudaError_t e = launch_outlier_flags(static_cast<const __half *>(X), M, K, tb, flags, L.flag_chunks, s))
+        return from_cuda(e);
+    QuantizeArgs q{};
+    q.X = static_cast<const __half *>(X);
+    q.M = M; q.K = K;
+    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
+    q.CA = CA; q.SCA = SCA; q.outlier_idx = outlier_idx; q.n_outliers = n_outliers;
+    q.kcap = L.kcap;
+    return from_cuda(launch_quantize(q, s));
+}
+
+int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                   const void *W_outlier, float threshold, const void *bias, void *Y, void *ws,
+                   size_t ws_bytes, void *stream) {
+    if (!X || !CB || !SCB || !Y || !ws) return INT8LT_ERR_NULL;
+    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (!aligned(X, 16) || !aligned(CB, 16) || !aligned(SCB, 4) || !aligned(Y, 16) || !aligned(ws, 16) ||
+        (W_outlier && !aligned(W_outlier, 16)) || (bias && !aligned(bias, 2)))
+        return INT8LT_ERR_ALIGN;
+    if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
+    const WsLayout L = ws_layout(M, N, K);
+    if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
+    if (M == 0 || N == 0) return INT8LT_OK;
+    if (int st = check_device()) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __half *x = static_cast<const __half *>(X);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    const uint16_t tb = threshold_bits(threshold);
+    uint32_t *flags = at<uint32_t>(ws, L.flags);
+    if (cudaError_t e = launch_outlier_flags(x, M, K, tb, flags, L.flag_chunks, s)) return from_cuda(e);
+
+    const bool decode = M <= kDecodeMaxM;
+    const int splits = decode ? gemv_splits(N, K) : 1;
+    QuantizeArgs q{};
+    q.X = x; q.M = M; q.K = K;
+    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
+    q.CA = at<int8_t>(ws, L.ca); q.SCA = at<float>(ws, L.sca);
+    q.outlier_idx = at<int32_t>(ws, L.idx); q.n_outliers = &hdr->n_outliers;
+    q.Xo = at<__half>(ws, L.xo); q.kcap = L.kcap;
+    q.W_outlier = static_cast<const __half *>(W_outlier); q.CB = CB; q.SCB = SCB; q.N = N;
+    if (!decode) q.Wo = at<__half>(ws, L.wo);
+    if (decode && splits > 1) {
+        q.acc = at<int32_t>(ws, L.acc); q.acc_words = N * 16;
+        q.cnt = at<uint32_t>(ws, L.cnt); q.cnt_words = ceil_div(N, 32);
+    }
+    if (cudaError_t e = launch_quantize(q, s)) return from_cuda(e);
+
+    if (decode) {
+        GemvArgs g{};
+        g.CA = q.CA; g.CB = CB; g.SCA = q.SCA; g.SCB = SCB;
+        g.Xo = q.Xo; g.kcap = L.kcap; g.outlier_idx = q.outlier_idx; g.n_outliers = q.n_outliers;
+        g.W_outlier = q.W_outlier; g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
+        g.acc = q.acc; g.cnt = q.cnt;
+        g.M = M; g.N = N; g.K = K; g.splits = splits;
+        return from_cuda(launch_gemv(g, s));
+    }
+    GemmArgs g{};
+    g.CA = q.CA; g.CB = CB; g.SCA = q.SCA; g.SCB = SCB;
+    g.Xo = q.Xo; g.Wo = q.Wo; g.kcap = L.kcap; g.n_outliers = q.n_outliers;
+    g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
+    g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    return from_cuda(launch_gemm_tc(g, s));
+}
+
+int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K, int32_t *C,
+                          void *ws, size_t ws_bytes, void *stream) {
+    if (!CA || !CB || !C || !ws) return INT8LT_ERR_NULL;
+    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (!aligned(CA, 16) || !aligned(CB, 16) || !aligned(C, 16) || !aligned(ws, 16)) return INT8LT_ERR_ALIGN;
+    const WsLayout L = ws_layout(M, N, K);
+    if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
+    if (M == 0 || N == 0) return INT8LT_OK;
+    if (int st = check_device()) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    if (M <= kDecodeMaxM) {
+        GemvArgs g{};
+        g.CA = CA; g.CB = CB; g.C32 = C;
+        g.M = M; g.N = N; g.K = K; g.splits = gemv_splits(N, K);
+        if (g.splits > 1) {
+            g.acc = at<int32_t>(ws, L.acc);
+            g.cnt = at<uint32_t>(ws, L.cnt);
+            if (cudaMemsetAsync(g.acc, 0, (size_t)N * 16 * 4, s) != cudaSuccess ||
+                cudaMemsetAsync(g.cnt, 0, (size_t)ceil_div(N, 32) * 4, s) != cudaSuccess)
+                return INT8LT_ERR_CUDA;
+        }
+        return from_cuda(launch_gemv(g, s));
+    }
+    GemmArgs g{};
+    g.CA = CA; g.CB = CB; g.C32 = C;
+    g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    return from_cuda(launch_gemm_tc(g, s));
+}
+
+int int8lt_debug_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream) {
+    if (!ws) return INT8LT_ERR_NULL;
+    if (ws_bytes < sizeof(WsHeader)) return INT8LT_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return INT8LT_ERR_ALIGN;
+    if (limit_ns < 1000 || limit_ns > 1000000000) return INT8LT_ERR_VALUE;
+    if (int st = check_device()) return st;
+    WsHeader *hdr = static_cast<WsHeader *>(ws);
+    return from_cuda(launch_wait_timeout(&hdr->status, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

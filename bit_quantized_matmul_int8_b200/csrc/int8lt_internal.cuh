@@ -1,0 +1,282 @@
+// Internal declarations of libint8lt: workspace layout, kernel launchers and
+// the sm_100a PTX wrappers (mbarrier, TMA, tcgen05) the kernels share.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/int8lt.h"
+
+namespace int8lt {
+
+constexpr int64_t kMaxK = 133144;       // 127^2 * K < 2^31
+constexpr int kDecodeMaxM = 16;         // M <= 16 takes the GEMV path
+constexpr int kColsPerFlagCta = 256;    // phase-A column strip (32 lanes x 8 fp16)
+constexpr int kMaxFlagChunks = 64;      // row chunks of phase A (partial bitmaps)
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every in-kernel wait
+
+// Device status bits (workspace header word 0).
+constexpr uint32_t kStatusTimeout = 1u;
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Byte offsets of the workspace sections (every section 1024-byte aligned).
+struct WsLayout {
+    int64_t M, N, K;
+    int64_t kwords;        // ceil(K / 32): words of one column bitmap
+    int64_t kcap;          // round_up(K, 64): row pitch (elements) of Xo / Wo
+    int64_t flag_chunks;   // phase-A row chunks actually used
+    size_t hdr, flags, idx, sca, ca, xo, wo, acc, cnt, total;
+};
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K);
+int64_t flag_chunks_for(int64_t M, int64_t K);
+
+// Workspace header (first 256 bytes).
+struct WsHeader {
+    uint32_t status;       // kStatus* bits, sticky until read
+    int32_t n_outliers;    // |O| of the last quantize pass
+    uint32_t pad[62];
+};
+
+// ------------------------------------------------------------- launchers --
+
+// fp16 bit pattern T: |x| >= threshold  <=>  (bits(x) & 0x7fff) >= T.
+uint16_t threshold_bits(float threshold);
+
+cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
+                                  cudaStream_t s);
+
+// Phase A: partial column-outlier bitmaps [flag_chunks][kwords].
+cudaError_t launch_outlier_flags(const __half *X, int64_t M, int64_t K, uint16_t tbits,
+                                 uint32_t *flags, int64_t flag_chunks, cudaStream_t s);
+
+struct QuantizeArgs {
+    const __half *X;
+    int64_t M, K;
+    const uint32_t *flags;
+    int64_t flag_chunks;
+    uint16_t tbits;
+    int8_t *CA;
+    float *SCA;
+    int32_t *outlier_idx;     // may be null
+    int32_t *n_outliers;      // may be null
+    __half *Xo;               // [M][kcap] or null
+    int64_t kcap;
+    // Outlier weight gather (M > 16 path): Wo[j][t] for t < round_up(|O|, 16).
+    const __half *W_outlier;  // null -> from CB/SCB
+    const int8_t *CB;
+    const float *SCB;
+    __half *Wo;               // [N][kcap] or null (no gather)
+    int64_t N;
+    // Split-K reduction buffers to clear (M <= 16 path), or null.
+    int32_t *acc;
+    int64_t acc_words;
+    uint32_t *cnt;
+    int64_t cnt_words;
+};
+cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
+
+struct GemmArgs {
+    const int8_t *CA;
+    const int8_t *CB;
+    const float *SCA;
+    const float *SCB;
+    const __half *Xo;         // [M][kcap]
+    const __half *Wo;         // [N][kcap]
+    int64_t kcap;
+    const int32_t *n_outliers;  // device; null -> no outlier term
+    const __half *bias;
+    __half *Y;
+    int32_t *C32;             // debug: raw int32 output instead of Y
+    int64_t M, N, K;
+    uint32_t *status;
+};
+cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
+
+struct GemvArgs {
+    const int8_t *CA;
+    const int8_t *CB;
+    const float *SCA;
+    const float *SCB;
+    const __half *Xo;           // [M][kcap]
+    int64_t kcap;
+    const int32_t *outlier_idx;
+    const int32_t *n_outliers;  // null -> no outlier term
+    const __half *W_outlier;    // null -> CB/SCB recovery
+    const __half *bias;
+    __half *Y;
+    int32_t *C32;               // debug: raw int32 output instead of Y
+    int32_t *acc;               // split-K partials [N][16]
+    uint32_t *cnt;              // split-K arrival counters [ceil(N/32)]
+    int64_t M, N, K;
+    int splits;
+};
+int gemv_splits(int64_t N, int64_t K);
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s);
+
+cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
+
+// ------------------------------------------------------- device helpers --
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the barrier phase with parity `parity` has completed, for at
+// most limit_ns. Returns false on timeout (the caller records it and stops).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void record_timeout(uint32_t *status) {
+    if (status) atomicOr(status, kStatusTimeout);
+}
+
+__device__ __forceinline__ void tma_prefetch(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 2-D tiled TMA load global -> shared, completion counted on `bar`.
+// x is the innermost (contiguous) coordinate in elements.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// --- tcgen05 (5th-generation tensor core, accumulators in tensor memory) ---
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, int8 x int8 -> int32.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, fp16 x fp16 -> fp32.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane
+// (base lane + t), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with
+// 128-byte swizzling: rows of 128 bytes, 8-row (1024-byte) swizzle atoms
+// stacked along M/N (stride byte offset 1024). Tile base 1024-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+    d |= (uint64_t)1 << 16;                    // leading byte offset (unused here)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset
+    d |= (uint64_t)1 << 46;                    // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
+#endif  // __CUDACC__
+
+}  // namespace int8lt

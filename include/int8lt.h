@@ -1,0 +1,169 @@
+/*
+ * int8lt -- LLM.int8() mixed-precision linear layer for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libint8lt.so. Computes Y = X W^T + bias the LLM.int8() way:
+ *
+ *   1. O = feature columns of X holding any |x| >= threshold (outliers);
+ *   2. the other columns of X are quantized row-wise (one absmax scale per
+ *      token), the weights per output channel (one absmax scale per row of W);
+ *   3. int8 x int8 GEMM with int32 accumulation on the tensor cores;
+ *   4. dequantize with the outer product of row and column scales;
+ *   5. add the fp16 product of the outlier columns (and the bias).
+ *
+ * Sources (web pages on LLM.int8(), cited by page title and section):
+ *   [HF]  "Hugging Face LLM.int8() integration into transformers and
+ *         accelerate" (agentlenshq.com): three-step recipe; absmax example;
+ *         Linear8bitLt / CB / SCB with W ~= CB * SCB / 127.
+ *   [P]   "LLM.int8() paper summary" (kurtkim.github.io/p/llm.int8/):
+ *         "8-bit Data Types and Quantization" (absmax equation);
+ *         "Int8 Matrix Multiplication with 16-bit Float Inputs and Outputs";
+ *         "Vector-wise Quantization"; "The Core of LLM.int8(): Mixed-precision
+ *         Decomposition" (threshold alpha = 6.0).
+ *
+ * Conventions for every entry point:
+ *   - Matrices are dense row-major. X is [M, K] (tokens x features), W and CB
+ *     are [N, K] (nn.Linear layout: one row per output channel), Y is [M, N].
+ *   - "fp16" means IEEE binary16, passed as void pointers. Every tensor
+ *     pointer is DEVICE memory owned by the caller; the library allocates
+ *     nothing and keeps no per-call state. `stream` is a cudaStream_t (NULL =
+ *     legacy default stream). All compute entry points are asynchronous and
+ *     stream-ordered; they return after the launches are queued.
+ *   - Host-side validation runs before any launch. On any error status no
+ *     kernel has been launched (except INT8LT_ERR_CUDA, reported when a
+ *     launch itself fails).
+ *   - Codes are int8 in [-127, 127]; scales are the fp32 absmax of the
+ *     quantized vector (not its reciprocal), so x ~= code * scale / 127.
+ *   - Shapes: M, N >= 0 (0 is a no-op returning INT8LT_OK), 16 <= K <= 133144
+ *     and K % 16 == 0 (int8 rows must be 16-byte multiples for the TMA
+ *     engine; 133144 * 127^2 < 2^31 keeps every int32 sum exact), N % 8 == 0.
+ *   - Alignment: X, W, W_outlier, CB, CA, Y and the workspace must be 16-byte
+ *     aligned; scale arrays 4-byte, bias 2-byte.
+ *   - NaN or infinite values inside X or W are outside the contract.
+ */
+#ifndef INT8LT_H
+#define INT8LT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    INT8LT_OK = 0,
+    INT8LT_ERR_NULL = 1,        /* a required pointer is NULL */
+    INT8LT_ERR_SHAPE = 2,       /* M, N or K outside the limits above */
+    INT8LT_ERR_ALIGN = 3,       /* a pointer is not aligned as required */
+    INT8LT_ERR_VALUE = 4,       /* threshold is NaN or negative */
+    INT8LT_ERR_WORKSPACE = 5,   /* ws_bytes < int8lt_workspace_size(...) */
+    INT8LT_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    INT8LT_ERR_TIMEOUT = 7,     /* a kernel gave up a bounded wait (device status) */
+    INT8LT_ERR_UNSUPPORTED = 8  /* current device is not compute capability 10.0 */
+} int8lt_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *int8lt_status_string(int status);
+
+/* Library version, as major * 10000 + minor * 100 + patch. */
+int int8lt_version(void);
+
+/*
+ * Workspace bytes that int8lt_forward needs for an [M, K] x [N, K]^T call.
+ * Holds the outlier bitmap partials, the outlier list and count, the device
+ * status word, CA/SCA, the gathered fp16 outlier activations, and either the
+ * gathered fp16 outlier weights (M > 16) or split-K int32 partials (M <= 16).
+ * The outlier buffers are sized for the worst case |O| = K, so any input fits.
+ * Returns 0 for shapes the library rejects.
+ */
+size_t int8lt_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Clear the workspace's device status word (stream-ordered). Call once after
+ * allocating a workspace; int8lt_read_device_status also clears it.
+ */
+int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronize `stream`, then read and clear the workspace's status word.
+ * Returns INT8LT_OK, or INT8LT_ERR_TIMEOUT if any kernel that used this
+ * workspace since the last read gave up a bounded wait (its outputs are then
+ * undefined), or INT8LT_ERR_CUDA if the stream reported an error.
+ */
+int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Weight conversion: W fp16 [N, K] -> CB int8 [N, K] and SCB fp32 [N].
+ * [HF] "transformers integration": weights become int8 in [-127, 127] with a
+ * per-output-channel scale, recoverable as W ~= CB * SCB / 127; [P] absmax
+ * equation, vector-wise (per output channel). SCB[j] = max_k |W[j,k]|,
+ * CB[j,k] = clamp(rint(W[j,k] * fp32(127 / SCB[j])), -127, 127) with the
+ * division and product rounded to fp32, ties to even; SCB[j] = 0 gives all
+ * zero codes. Deterministic and idempotent: re-running it gives identical
+ * bytes. K % 16 == 0 is not required here (K >= 1).
+ */
+int int8lt_prepare_weight(const void *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
+                          void *stream);
+
+/*
+ * Outlier detection and row-wise quantization of X fp16 [M, K].
+ * [HF] recipe step 1 and [P] "Mixed-precision Decomposition": O = { h : some
+ * |X[i,h]| >= threshold }, compared in fp32. [HF] step 2 and [P] absmax /
+ * vector-wise equations: for every row i, SCA[i] = max over h not in O of
+ * |X[i,h]|, CA[i,h] = clamp(rint(X[i,h] * fp32(127 / SCA[i])), -127, 127) for
+ * h not in O and CA[i,h] = 0 for h in O. threshold = +inf gives O empty;
+ * threshold = 0 puts every column in O.
+ *   outlier_idx: int32 [K] capacity; receives O in ascending order.
+ *   n_outliers : one int32 (device) receiving |O|.
+ *   ws         : scratch of at least int8lt_workspace_size(M, 8, K) bytes.
+ */
+int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold,
+                         int8_t *CA, float *SCA, int32_t *outlier_idx, int32_t *n_outliers,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The LLM.int8() forward: Y fp16 [M, N] =
+ *     fp16( C[i,j] * SCA[i] * SCB[j] / 127^2 + sum_{h in O} X[i,h] Wo[j,h] + bias[j] )
+ * with C = CA CB^T accumulated exactly in int32 ([P] int8 matmul and
+ * vector-wise equations), O and CA/SCA as in int8lt_quantize_rows, and the
+ * outlier term of [P] "Mixed-precision Decomposition" / [HF] step 3.
+ * The combination is computed in fp32 and rounded once to fp16.
+ *   CB, SCB   : from int8lt_prepare_weight.
+ *   W_outlier : fp16 [N, K] weights for the outlier columns (only the columns
+ *               in O are read), or NULL to use fp16(fp32(CB * SCB) / 127).
+ *   bias      : fp16 [N] or NULL.
+ *   ws        : at least int8lt_workspace_size(M, N, K) bytes.
+ * Dispatch: M <= 16 runs the memory-bound split-K GEMV; larger M runs the
+ * tcgen05 int8 GEMM with the outlier MMA and the dequantization fused into it.
+ */
+int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K,
+                   const int8_t *CB, const float *SCB, const void *W_outlier,
+                   float threshold, const void *bias, void *Y,
+                   void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- tests -- */
+
+/*
+ * Test entry: the int8 GEMM alone, C int32 [M, N] = CA [M, K] . CB [N, K]^T,
+ * through the same kernels int8lt_forward dispatches to (M <= 16: the GEMV,
+ * otherwise the tcgen05 GEMM) with the dequantizing epilogue replaced by an
+ * int32 store, so the accumulators can be compared bit for bit. Same shape,
+ * alignment and workspace rules as int8lt_forward.
+ */
+int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K,
+                          int32_t *C, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Test entry: launch one block that waits on a barrier nothing ever arrives
+ * at, with the same bounded-wait routine the GEMM pipeline uses, limited to
+ * `limit_ns` nanoseconds (1e3 .. 1e9). The kernel records INT8LT_ERR_TIMEOUT
+ * in the workspace status word and returns normally; no GPU fault, trap or
+ * hang is involved.
+ */
+int int8lt_debug_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT8LT_H */

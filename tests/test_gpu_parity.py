@@ -1,0 +1,234 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Integer stages (outlier set, CA/SCA, CB/SCB, int32 accumulators) must be
+bit-exact; the fp16 output must satisfy |dY| <= 2e-3 * max(1, |y|) against
+the oracle's fp64 value. Shapes span several 128 x 256 tiles with ragged tails.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_matmul_int8_b200 import _lib
+from bit_quantized_matmul_int8_b200 import workloads as wl
+from gpu_common import case_inputs, check_y, dev, ensure_built, host, run_forward
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    ensure_built()
+
+
+# ------------------------------------------------------------ weight prep --
+
+@pytest.mark.parametrize("N,K", [(64, 64), (200, 4096), (24, 40), (8, 3), (513, 1000)])
+def test_prepare_weight_bit_exact(N, K):
+    w = wl.random_case(31, 4, K, N)
+    W = wl.make_w(w)
+    W[N // 2] = 0                                   # all-zero channel: scale 0
+    CB, SCB = _lib.int8lt_prepare_weight(dev(W))
+    CBo, SCBo = oracle.prepare_weight(W)
+    assert np.array_equal(host(CB), CBo)
+    assert np.array_equal(host(SCB).view(np.uint32), SCBo.view(np.uint32))
+
+
+def test_prepare_weight_idempotent():
+    W = dev(wl.make_w(wl.random_case(32, 4, 256, 96)))
+    a = [t.clone() for t in _lib.int8lt_prepare_weight(W)]
+    b = _lib.int8lt_prepare_weight(W)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---------------------------------------------------------- quantize rows --
+
+QCASES = [
+    ("tiny", wl.WORKLOADS["tiny_16x64x64"], None),
+    ("ragged", wl.random_case(41, 37, 96, 8, n_outliers=5, frac=0.3), None),
+    ("wide", wl.random_case(42, 130, 4112, 8, n_outliers=9, frac=0.75), None),
+    ("many_rows", wl.random_case(43, 3000, 256, 8, n_outliers=3, frac=0.01), None),
+    ("no_outliers", wl.random_case(44, 64, 512, 8, n_outliers=0), None),
+]
+
+
+@pytest.mark.parametrize("name,w,_", QCASES, ids=[c[0] for c in QCASES])
+@pytest.mark.parametrize("thr", [None, math.inf, 0.0, 1.5])
+def test_quantize_rows_bit_exact(name, w, _, thr):
+    X = wl.make_x(w)
+    t = w.threshold if thr is None else thr
+    CA, SCA, idx = _lib.int8lt_quantize_rows(dev(X), t)
+    CAo, SCAo, idxo = oracle.quantize_rows(X, t)
+    assert np.array_equal(host(idx), idxo)
+    assert np.array_equal(host(CA), CAo)
+    assert np.array_equal(host(SCA).view(np.uint32), SCAo.view(np.uint32))
+    if thr is None:
+        assert host(idx).tolist() == wl.outlier_columns(w).tolist()
+
+
+def test_quantize_threshold_boundary():
+    X = np.zeros((40, 64), np.float16)
+    X[3, 5] = 6.0
+    X[7, 9] = np.float16(5.99609375)
+    X[30, 60] = -6.0
+    X[11, 33] = 65504.0
+    X[:, 0] = np.linspace(-1, 1, 40)
+    CA, SCA, idx = _lib.int8lt_quantize_rows(dev(X), 6.0)
+    assert host(idx).tolist() == [5, 33, 60]
+    CAo, SCAo, _ = oracle.quantize_rows(X, 6.0)
+    assert np.array_equal(host(CA), CAo) and np.array_equal(host(SCA), SCAo)
+
+
+def test_quantize_empty_batch():
+    X = torch.empty((0, 64), dtype=torch.float16, device="cuda")
+    CA, SCA, idx = _lib.int8lt_quantize_rows(X, 6.0)
+    assert CA.shape == (0, 64) and len(idx) == 0
+
+
+# ------------------------------------------------------------ int32 GEMM --
+
+GEMM_SHAPES = [(128, 256, 128), (300, 520, 400), (129, 264, 4112), (1000, 776, 2048),
+               (17, 8, 16), (1, 64, 64), (4, 1000, 512), (16, 4096, 1024), (3, 40, 48),
+               (4, 38400, 256), (16, 8, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_int32_bit_exact(M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    if M > 2:
+        A[1] = 127
+        B[0] = -127 if N > 1 else B[0]
+    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    ref = A.astype(np.int64) @ B.astype(np.int64).T          # exact in int64
+    assert np.array_equal(C.astype(np.int64), ref)
+
+
+def test_gemm_int32_matches_oracle_routine():
+    rng = np.random.default_rng(9)
+    A = rng.integers(-127, 128, (200, 336), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-127, 128, (264, 336), dtype=np.int64).astype(np.int8)
+    assert np.array_equal(host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B))), oracle.gemm_i32(A, B))
+
+
+def test_gemm_int32_extreme_k():
+    # K near the int32 limit: 127 * 127 * K stays below 2^31
+    K = 133136
+    A = np.full((20, K), 127, np.int8)
+    B = np.full((8, K), -127, np.int8)
+    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    assert (C.astype(np.int64) == -127 * 127 * K).all()
+
+
+# --------------------------------------------------------------- forward --
+
+FCASES = [
+    wl.WORKLOADS["tiny_16x64x64"],
+    wl.random_case(51, 300, 512, 264, n_outliers=4, frac=0.5),
+    wl.random_case(52, 129, 1040, 520, n_outliers=7, frac=0.75, has_bias=False),
+    wl.random_case(53, 17, 256, 40, n_outliers=2),             # smallest prefill M
+    wl.random_case(54, 1, 1024, 2048, n_outliers=3, frac=1.0),  # decode
+    wl.random_case(55, 4, 768, 312, n_outliers=6, frac=1.0),
+    wl.random_case(56, 16, 4096, 1024, n_outliers=6, frac=1.0, has_bias=False),
+    wl.random_case(57, 600, 2048, 1024, n_outliers=70, frac=0.2),  # > 64 outliers
+    wl.random_case(58, 200, 384, 136, n_outliers=0),
+]
+
+
+@pytest.mark.parametrize("w", FCASES, ids=[w.name for w in FCASES])
+@pytest.mark.parametrize("thr", ["cfg", "inf"])
+def test_forward_vs_oracle(w, thr):
+    t = w.threshold if thr == "cfg" else math.inf
+    X, W, b = case_inputs(w)
+    Yg, Y64 = run_forward(X, W, b, t)
+    check_y(Yg, Y64, w.name)
+
+
+@pytest.mark.parametrize("w", [FCASES[1], FCASES[4], FCASES[7]], ids=lambda w: w.name)
+def test_forward_int8_outlier_weights(w):
+    """W_outlier = NULL: outlier weights come from CB * SCB / 127."""
+    X, W, b = case_inputs(w)
+    Yg, Y64 = run_forward(X, W, b, w.threshold, keep_w=False)
+    check_y(Yg, Y64, w.name)
+
+
+@pytest.mark.parametrize("M", [1, 16, 200])
+def test_forward_all_columns_outlier(M):
+    """threshold 0: every column is an outlier, the layer is an fp16 matmul."""
+    w = wl.random_case(60 + M, M, 192, 136, n_outliers=2)
+    X, W, b = case_inputs(w)
+    X[X == 0] = np.float16(1e-3)
+    Yg, Y64 = run_forward(X, W, b, 0.0)
+    check_y(Yg, Y64, "all-outlier")
+    ref = X.astype(np.float64) @ W.astype(np.float64).T + b.astype(np.float64)
+    check_y(Yg, ref, "all-outlier vs fp64 matmul")
+
+
+def test_forward_deterministic_and_reuses_workspace():
+    w = FCASES[1]
+    X, W, b = case_inputs(w)
+    Xd, Wd, bd = dev(X), dev(W), dev(b)
+    CB, SCB = _lib.int8lt_prepare_weight(Wd)
+    ws = _lib.workspace(w.M, w.N, w.K)
+    y1 = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, ws=ws).clone()
+    # a call with a different outlier set in between must not leak into the next
+    X2 = X.copy()
+    X2[:, 7] = 50.0
+    _lib.int8lt_forward(dev(X2), CB, SCB, Wd, 6.0, bd, ws=ws)
+    y2 = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert _lib.int8lt_read_device_status(ws) == 0
+
+
+def test_forward_empty_batch():
+    W = dev(wl.make_w(wl.random_case(70, 1, 64, 64)))
+    CB, SCB = _lib.int8lt_prepare_weight(W)
+    X = torch.empty((0, 64), dtype=torch.float16, device="cuda")
+    Y = _lib.int8lt_forward(X, CB, SCB, W, 6.0)
+    assert Y.shape == (0, 64)
+
+
+def test_forward_on_side_stream():
+    w = FCASES[1]
+    X, W, b = case_inputs(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        Xd, Wd, bd = dev(X), dev(W), dev(b)
+        CB, SCB = _lib.int8lt_prepare_weight(Wd, stream=s)
+        Y = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, stream=s)
+    s.synchronize()
+    CBo, SCBo = oracle.prepare_weight(W)
+    Y64, _, _ = oracle.forward(X, CBo, SCBo, W, 6.0, b)
+    check_y(host(Y), Y64, "side stream")
+
+
+# ------------------------------------------------------- failure detection --
+
+def test_bounded_wait_reports_timeout():
+    ws = _lib.workspace(32, 64, 64)
+    assert _lib.int8lt_read_device_status(ws) == 0
+    _lib.int8lt_debug_wait_timeout(ws, 1_000_000)          # 1 ms, nothing arrives
+    assert _lib.int8lt_read_device_status(ws) == _lib.STATUS_CODE["INT8LT_ERR_TIMEOUT"]
+    assert _lib.int8lt_read_device_status(ws) == 0           # the read cleared it
+    # the context is still usable
+    X = dev(wl.make_x(wl.WORKLOADS["tiny_16x64x64"]))
+    CA, SCA, idx = _lib.int8lt_quantize_rows(X, 6.0)
+    torch.cuda.synchronize()
+    assert len(idx) == 2
+
+
+def test_validation_errors_raise():
+    W = dev(wl.make_w(wl.random_case(71, 1, 64, 64)))
+    CB, SCB = _lib.int8lt_prepare_weight(W)
+    X = dev(wl.make_x(wl.random_case(71, 32, 64, 64)))
+    with pytest.raises(_lib.Int8ltError) as e:
+        _lib.int8lt_forward(X, CB, SCB, W, float("nan"))
+    assert e.value.name == "INT8LT_ERR_VALUE"
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(_lib.Int8ltError) as e:
+        _lib.int8lt_forward(X, CB, SCB, W, 6.0, ws=ws)
+    assert e.value.name == "INT8LT_ERR_WORKSPACE"
