@@ -158,9 +158,10 @@ int int8lt_prepare_weight(const void *W, int64_t N, int64_t K, int8_t *CB, float
 
 int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold, int8_t *CA, float *SCA,
                          int32_t *outlier_idx, int32_t *n_outliers, void *ws, size_t ws_bytes, void *stream) {
-    if (!X || !CA || !SCA || !outlier_idx || !n_outliers || !ws) return INT8LT_ERR_NULL;
     if (!shape_ok(M, 8, K)) return INT8LT_ERR_SHAPE;
-    if (!aligned(X, 16) || !aligned(CA, 16) || !aligned(SCA, 4) || !aligned(outlier_idx, 4) ||
+    if (!n_outliers || !ws) return INT8LT_ERR_NULL;
+    if (M > 0 && (!X || !CA || !SCA || !outlier_idx)) return INT8LT_ERR_NULL;
+    if ((M > 0 && (!aligned(X, 16) || !aligned(CA, 16) || !aligned(SCA, 4) || !aligned(outlier_idx, 4))) ||
         !aligned(n_outliers, 4) || !aligned(ws, 16))
         return INT8LT_ERR_ALIGN;
     if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
@@ -189,15 +190,15 @@ int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold, i
 int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
                    const void *W_outlier, float threshold, const void *bias, void *Y, void *ws,
                    size_t ws_bytes, void *stream) {
-    if (!X || !CB || !SCB || !Y || !ws) return INT8LT_ERR_NULL;
     if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (M == 0 || N == 0) return INT8LT_OK;  // empty output: nothing to read or write
+    if (!X || !CB || !SCB || !Y || !ws) return INT8LT_ERR_NULL;
     if (!aligned(X, 16) || !aligned(CB, 16) || !aligned(SCB, 4) || !aligned(Y, 16) || !aligned(ws, 16) ||
         (W_outlier && !aligned(W_outlier, 16)) || (bias && !aligned(bias, 2)))
         return INT8LT_ERR_ALIGN;
     if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
     const WsLayout L = ws_layout(M, N, K);
     if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
-    if (M == 0 || N == 0) return INT8LT_OK;
     if (int st = check_device()) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const __half *x = static_cast<const __half *>(X);
@@ -241,12 +242,12 @@ int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K, const int8_t 
 
 int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K, int32_t *C,
                           void *ws, size_t ws_bytes, void *stream) {
-    if (!CA || !CB || !C || !ws) return INT8LT_ERR_NULL;
     if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (M == 0 || N == 0) return INT8LT_OK;
+    if (!CA || !CB || !C || !ws) return INT8LT_ERR_NULL;
     if (!aligned(CA, 16) || !aligned(CB, 16) || !aligned(C, 16) || !aligned(ws, 16)) return INT8LT_ERR_ALIGN;
     const WsLayout L = ws_layout(M, N, K);
     if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
-    if (M == 0 || N == 0) return INT8LT_OK;
     if (int st = check_device()) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);

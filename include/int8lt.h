@@ -28,7 +28,9 @@
  *     nothing and keeps no per-call state. `stream` is a cudaStream_t (NULL =
  *     legacy default stream). All compute entry points are asynchronous and
  *     stream-ordered; they return after the launches are queued.
- *   - Host-side validation runs before any launch. On any error status no
+ *   - Host-side validation runs before any launch. A call whose output is
+ *     empty (M == 0 or N == 0, with a valid K) returns INT8LT_OK without
+ *     reading its pointers, which may then be NULL. On any error status no
  *     kernel has been launched (except INT8LT_ERR_CUDA, reported when a
  *     launch itself fails).
  *   - Codes are int8 in [-127, 127]; scales are the fp32 absmax of the
