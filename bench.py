@@ -1,0 +1,444 @@
+"""Benchmark of the LLM.int8() linear layer on B200.
+
+A step is one int8lt_forward (outlier detect + row quantize + int8 tensor-core
+GEMM with the fused dequantize / fp16 outlier product / bias epilogue) over
+the 6.7B-class projection prefill X fp16 [2048 x 4096] . W [4096 x 4096]^T
+with 6 outlier feature columns (threshold 6.0) unless --workload says
+otherwise. Inputs are resident in HBM; several input sets rotate so that the
+bytes touched between two uses of a set exceed the 126 MB L2.
+
+Prints ONE JSON line (rank 0). Value = effective TOPS = 2*M*N*K per forward,
+summed over ranks, over the max-over-ranks device time of the timed steps.
+Multi-GPU: one process per GPU, each runs its own replica (independent
+batches, no collective on the data path); NCCL only for the barrier and the
+max-over-ranks time.
+
+--impl reference times the CPU oracle (plain single-threaded C) on a bounded
+sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from bit_quantized_matmul_int8_b200 import workloads as wl  # noqa: E402
+
+METRIC = "int8 mixed-precision linear effective TOPS & tokens/s; % of INT8 peak / HBM BW"
+L2_BYTES = 126 * 1024 * 1024
+INT8_PER_BF16 = 2.0  # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s nominal)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--out", default=None, help="also append the JSON line to this file")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ peaks --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def dram_traffic(kernel_key: str, source_files: list[str]):
+    """Per-launch DRAM bytes from a committed ncu capture, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel_key)
+    if not d:
+        return None
+    h = hashlib.sha256()
+    for s in source_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    if d.get("source_sha256") != h.hexdigest():
+        return None
+    return float(d["bytes_per_launch"]) * d.get("scale", 1.0)
+
+
+# ----------------------------------------------------------------- clocks --
+
+NVML_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons via NVML while running."""
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = None
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                ids = vis.split(",")
+                if index < len(ids) and not ids[index].strip().isdigit():
+                    uuid = ids[index].strip()
+                elif index < len(ids):
+                    index = int(ids[index])
+            self.h = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid
+                      else pynvml.nvmlDeviceGetHandleByIndex(index))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than fail the bench
+            self.err = repr(e)
+
+    def _sample(self):
+        mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        try:
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(mhz)
+        self.reasons |= int(r)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        names = [n for bit, n in NVML_REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(self.samples), "source": "nvml"}
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+def cpu_oracle_sample(w: wl.Workload, target_s: float, X=None, W=None):
+    """Time the oracle forward on the first r rows of the workload (r sized to target_s)."""
+    import oracle
+
+    if X is None:
+        X = wl.make_x(w)
+    if W is None:
+        W = wl.make_w(w)
+    b = wl.make_bias(w)
+    CB, SCB = oracle.prepare_weight(W)       # weight conversion: offline, not timed
+    probe = min(w.M, 8)
+    t0 = time.perf_counter()
+    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(probe))
+    per_row = (time.perf_counter() - t0) / probe          # upper bound: includes fixed costs
+    rows = int(max(1, min(w.M, target_s / max(per_row, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(rows))
+    dt = time.perf_counter() - t0
+    ops = 2.0 * rows * w.N * w.K
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {w.M} rows x all {w.N} output channels (outlier set over "
+                      f"all rows, row quantize, int64-checked int8 GEMM, fp64 dequant + outlier "
+                      f"product); {dt:.2f} s on 1 host core",
+            "host_cores": os.cpu_count(), "seconds": dt, "rows": rows}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    import oracle
+
+    X, W = wl.make_x(w), wl.make_w(w)
+    b = wl.make_bias(w)
+    CB, SCB = oracle.prepare_weight(W)
+    t0 = time.perf_counter()
+    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(1))
+    t_row = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)      # whole run ~ 2.5 minutes
+    rows = int(max(1, min(w.M, budget / max(t_row, 1e-6))))
+    for _ in range(args.warmup):
+        oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(rows))
+    times = []
+    for s in range(args.steps):
+        r0 = (s * rows) % max(1, w.M - rows + 1)
+        t0 = time.perf_counter()
+        oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(r0, r0 + rows))
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    ops = 2.0 * rows * w.N * w.K * args.steps
+    value = ops / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "n_outliers": w.n_outliers,
+                   "threshold": w.threshold, "rows_per_step": rows},
+        "tokens_per_s": rows * args.steps / total,
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} of {w.M} rows per step, all {w.N} output channels"},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    emit(line, args.out)
+
+
+def emit(line: dict, out: str | None):
+    s = json.dumps(line)
+    print(s, flush=True)
+    if out:
+        with open(out, "a") as f:
+            f.write(s + "\n")
+
+
+# -------------------------------------------------------------- GPU bench --
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+
+    from bit_quantized_matmul_int8_b200 import _lib, build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[args.workload]
+    M, N, K = w.M, w.N, w.K
+    peaks = load_peaks()
+
+    X = wl.make_x(w)
+    W = wl.make_w(w)
+    b = wl.make_bias(w)
+    Xh = torch.from_numpy(X).pin_memory()
+    Wd = torch.from_numpy(W).to(dev)
+    bd = torch.from_numpy(b).to(dev) if b is not None else None
+    CB0, SCB = _lib.int8lt_prepare_weight(Wd)
+    torch.cuda.synchronize()
+
+    # Rotating input sets: X, CB, Y and workspace per set.
+    ws_bytes = _lib.int8lt_workspace_size(M, N, K)
+    touched = X.nbytes + M * K + (M * N * 2) + M * K + N * K  # X + CA + Y + CB(+CA write)
+    R = int(min(16, max(3, math.ceil(3 * L2_BYTES / touched))))
+    Xs = [Xh.to(dev) for _ in range(R)]
+    CBs = [CB0.clone() for _ in range(R)]
+    Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(R)]
+    WSs = [_lib.workspace(M, N, K, dev) for _ in range(R)]
+    del CB0
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        r = s % R
+        _lib.int8lt_forward(Xs[r], CBs[r], SCB, Wd, w.threshold, bd, Ys[r], WSs[r], stream)
+
+    for s in range(max(3, args.warmup)):
+        step(s)
+    torch.cuda.synchronize()
+
+    # One CUDA graph per timed step, each with external event-record nodes
+    # around the quantize half and the matmul half of the forward.
+    decode = M <= 16
+    K_steps = args.steps
+    evq = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K_steps)]
+    evm = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K_steps)]
+    eve = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K_steps)]
+    graphs = []
+    cap_stream = torch.cuda.Stream(device=dev)
+    for s in range(K_steps):
+        r = s % R
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            cs = torch.cuda.current_stream()
+            evq[s].record(cs)
+            _lib.int8lt_forward_quantize(Xs[r], CBs[r], SCB, Wd, w.threshold, WSs[r], cs)
+            evm[s].record(cs)
+            _lib.int8lt_forward_matmul(M, CBs[r], SCB, Wd, bd, Ys[r], WSs[r], cs)
+            eve[s].record(cs)
+        graphs.append(g)
+    for g in graphs[: min(len(graphs), max(3, args.warmup))]:
+        g.replay()
+    torch.cuda.synchronize()
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        t_start.record()
+        for g in graphs:
+            g.replay()
+        t_end.record()
+        torch.cuda.synchronize()
+    if dist:
+        tdist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    q_ms = [evq[s].elapsed_time(evm[s]) for s in range(K_steps)]
+    m_ms = [evm[s].elapsed_time(eve[s]) for s in range(K_steps)]
+    if dist:
+        t = torch.tensor([elapsed_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    for ws in WSs:
+        st = _lib.int8lt_read_device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {_lib.STATUS.get(st)} after the timed steps")
+
+    ops = 2.0 * M * N * K
+    value = ops * K_steps * world / (elapsed_ms * 1e-3) / 1e12
+    tokens_per_s = M * K_steps * world / (elapsed_ms * 1e-3)
+
+    # Roofline of the dominant kernel: the matmul half is one launch (GEMM or GEMV).
+    m_avg = statistics.mean(m_ms) * 1e-3
+    q_avg = statistics.mean(q_ms) * 1e-3
+    src = ["bit_quantized_matmul_int8_b200/csrc/gemm_tc.cu" if not decode
+           else "bit_quantized_matmul_int8_b200/csrc/gemv.cu",
+           "bit_quantized_matmul_int8_b200/csrc/int8lt_internal.cuh"]
+    kname = ("gemm_i8_kernel" if not decode else "gemv_i8_kernel") + "@" + w.name
+    traffic = dram_traffic(kname, src)
+    if not decode:
+        peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        achieved = ops / m_avg / 1e12
+        roof = {"bound": "tensor", "kernel": "gemm_i8_kernel", "achieved": achieved, "peak": peak,
+                "unit": "TOPS", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 2 "
+                               f"(int8/bf16 nominal ratio)",
+                "algorithmic_units": f"2*M*N*K = {ops:.4g} int8 ops per launch"}
+    else:
+        n_out = w.n_outliers if math.isfinite(w.threshold) else 0
+        alg_bytes = N * K + 4 * N + M * K + 4 * M + 2 * M * N + 2 * M * n_out + 2 * N * n_out
+        achieved = alg_bytes / m_avg / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": "gemv_i8_kernel", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peaks['source']} HBM copy",
+                "algorithmic_units": f"{alg_bytes} bytes per launch (CB + SCB + CA + SCA + Y + outliers)"}
+
+    # End to end through the public API: pinned X -> device, forward, Y -> pinned host.
+    Yh = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    layer_ws = WSs[0]
+    Xd = torch.empty_like(Xs[0])
+    Yd = torch.empty_like(Ys[0])
+    for _ in range(3):
+        Xd.copy_(Xh, non_blocking=True)
+        _lib.int8lt_forward(Xd, CBs[0], SCB, Wd, w.threshold, bd, Yd, layer_ws, stream)
+        Yh.copy_(Yd, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = min(K_steps, 100)
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n_e2e):
+        Xd.copy_(Xh, non_blocking=True)
+        _lib.int8lt_forward(Xd, CBs[0], SCB, Wd, w.threshold, bd, Yd, layer_ws, stream)
+        Yh.copy_(Yd, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": ops * n_e2e * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
+           "steps": n_e2e, "tokens_per_s": M * n_e2e * world / (e2e_ms * 1e-3)}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": w.name, "M": M, "K": K, "N": N, "n_outliers": w.n_outliers,
+                   "threshold": w.threshold, "x": "N(0,1) fp16 + planted outlier columns",
+                   "w": f"N(0,{w.sigma_w}) fp16", "l2": f"{R} rotating input sets "
+                   f"({R * touched / 2**20:.0f} MiB touched per cycle) > 126 MB L2",
+                   "parallelism": f"replicas x{world}", "cuda_graphs": True},
+        "tokens_per_s": tokens_per_s,
+        "phases_ms": {"quantize": q_avg * 1e3, "matmul": m_avg * 1e3},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": K_steps * 3,
+        "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W)
+    elif not args.no_cpu_baseline:
+        line["cpu_baseline"] = None
+    emit(line, args.out)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -26,7 +26,8 @@ STATUS_CODE = {v: k for k, v in STATUS.items()}
 EXPORTS = [
     "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
-    "int8lt_forward", "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
+    "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
+    "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
 ]
 
 
@@ -50,6 +51,8 @@ _SIGS = {
     "int8lt_prepare_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
     "int8lt_quantize_rows": (ctypes.c_int, [_P, _I64, _I64, _F, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8lt_forward": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P, _SZ, _P]),
+    "int8lt_forward_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _SZ, _P]),
+    "int8lt_forward_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
 }
@@ -183,6 +186,28 @@ def int8lt_forward(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
            lib().int8lt_forward(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier),
                                 float(threshold), _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(),
                                 _stream(stream)))
+    return Y
+
+
+def int8lt_forward_quantize(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                            W_outlier: torch.Tensor | None, threshold: float, ws: torch.Tensor,
+                            stream=None) -> None:
+    """First half of int8lt_forward: quantize X (and gather outlier weights) into ws."""
+    M, K = X.shape
+    N = CB.shape[0]
+    _check("int8lt_forward_quantize",
+           lib().int8lt_forward_quantize(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier),
+                                         float(threshold), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def int8lt_forward_matmul(M: int, CB: torch.Tensor, SCB: torch.Tensor,
+                          W_outlier: torch.Tensor | None, bias: torch.Tensor | None,
+                          Y: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """Second half of int8lt_forward: GEMM/GEMV + fused epilogue from ws into Y."""
+    N, K = CB.shape
+    _check("int8lt_forward_matmul",
+           lib().int8lt_forward_matmul(M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier), _ptr(bias),
+                                       _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
     return Y
 
 

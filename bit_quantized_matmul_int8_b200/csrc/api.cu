@@ -102,6 +102,74 @@ cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_
 }
 }  // namespace int8lt
 
+namespace {
+
+// Host-side checks shared by the forward entry points.
+int check_forward_args(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                       const void *W_outlier, float threshold, const void *bias, const void *Y, bool need_x,
+                       bool need_y, void *ws, size_t ws_bytes) {
+    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (M == 0 || N == 0) return -1;  // empty output: nothing to read or write
+    if ((need_x && !X) || !CB || !SCB || (need_y && !Y) || !ws) return INT8LT_ERR_NULL;
+    if ((need_x && !aligned(X, 16)) || !aligned(CB, 16) || !aligned(SCB, 4) || (need_y && !aligned(Y, 16)) ||
+        !aligned(ws, 16) || (W_outlier && !aligned(W_outlier, 16)) || (bias && !aligned(bias, 2)))
+        return INT8LT_ERR_ALIGN;
+    if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
+    if (ws_bytes < ws_layout(M, N, K).total) return INT8LT_ERR_WORKSPACE;
+    return check_device();
+}
+
+int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                     const void *W_outlier, float threshold, void *ws, cudaStream_t s) {
+    const WsLayout L = ws_layout(M, N, K);
+    const __half *x = static_cast<const __half *>(X);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    const uint16_t tb = threshold_bits(threshold);
+    uint32_t *flags = at<uint32_t>(ws, L.flags);
+    if (cudaError_t e = launch_outlier_flags(x, M, K, tb, flags, L.flag_chunks, s)) return from_cuda(e);
+    const bool decode = M <= kDecodeMaxM;
+    const int splits = decode ? gemv_splits(N, K) : 1;
+    QuantizeArgs q{};
+    q.X = x; q.M = M; q.K = K;
+    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
+    q.CA = at<int8_t>(ws, L.ca); q.SCA = at<float>(ws, L.sca);
+    q.outlier_idx = at<int32_t>(ws, L.idx); q.n_outliers = &hdr->n_outliers;
+    q.Xo = at<__half>(ws, L.xo); q.kcap = L.kcap;
+    q.W_outlier = static_cast<const __half *>(W_outlier); q.CB = CB; q.SCB = SCB; q.N = N;
+    if (!decode) q.Wo = at<__half>(ws, L.wo);
+    if (decode && splits > 1) {
+        q.acc = at<int32_t>(ws, L.acc); q.acc_words = N * 16;
+        q.cnt = at<uint32_t>(ws, L.cnt); q.cnt_words = ceil_div(N, 32);
+    }
+    return from_cuda(launch_quantize(q, s));
+}
+
+int forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB, const void *W_outlier,
+                   const void *bias, void *Y, void *ws, cudaStream_t s) {
+    const WsLayout L = ws_layout(M, N, K);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    if (M <= kDecodeMaxM) {
+        const int splits = gemv_splits(N, K);
+        GemvArgs g{};
+        g.CA = at<int8_t>(ws, L.ca); g.CB = CB; g.SCA = at<float>(ws, L.sca); g.SCB = SCB;
+        g.Xo = at<__half>(ws, L.xo); g.kcap = L.kcap;
+        g.outlier_idx = at<int32_t>(ws, L.idx); g.n_outliers = &hdr->n_outliers;
+        g.W_outlier = static_cast<const __half *>(W_outlier); g.bias = static_cast<const __half *>(bias);
+        g.Y = static_cast<__half *>(Y);
+        if (splits > 1) { g.acc = at<int32_t>(ws, L.acc); g.cnt = at<uint32_t>(ws, L.cnt); }
+        g.M = M; g.N = N; g.K = K; g.splits = splits;
+        return from_cuda(launch_gemv(g, s));
+    }
+    GemmArgs g{};
+    g.CA = at<int8_t>(ws, L.ca); g.CB = CB; g.SCA = at<float>(ws, L.sca); g.SCB = SCB;
+    g.Xo = at<__half>(ws, L.xo); g.Wo = at<__half>(ws, L.wo); g.kcap = L.kcap; g.n_outliers = &hdr->n_outliers;
+    g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
+    g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    return from_cuda(launch_gemm_tc(g, s));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *int8lt_status_string(int status) {
@@ -190,54 +258,27 @@ int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold, i
 int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
                    const void *W_outlier, float threshold, const void *bias, void *Y, void *ws,
                    size_t ws_bytes, void *stream) {
-    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
-    if (M == 0 || N == 0) return INT8LT_OK;  // empty output: nothing to read or write
-    if (!X || !CB || !SCB || !Y || !ws) return INT8LT_ERR_NULL;
-    if (!aligned(X, 16) || !aligned(CB, 16) || !aligned(SCB, 4) || !aligned(Y, 16) || !aligned(ws, 16) ||
-        (W_outlier && !aligned(W_outlier, 16)) || (bias && !aligned(bias, 2)))
-        return INT8LT_ERR_ALIGN;
-    if (std::isnan(threshold) || threshold < 0.f) return INT8LT_ERR_VALUE;
-    const WsLayout L = ws_layout(M, N, K);
-    if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
-    if (int st = check_device()) return st;
+    int st = check_forward_args(X, M, N, K, CB, SCB, W_outlier, threshold, bias, Y, true, true, ws, ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const __half *x = static_cast<const __half *>(X);
-    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
-    const uint16_t tb = threshold_bits(threshold);
-    uint32_t *flags = at<uint32_t>(ws, L.flags);
-    if (cudaError_t e = launch_outlier_flags(x, M, K, tb, flags, L.flag_chunks, s)) return from_cuda(e);
+    if ((st = forward_quantize(X, M, N, K, CB, SCB, W_outlier, threshold, ws, s))) return st;
+    return forward_matmul(M, N, K, CB, SCB, W_outlier, bias, Y, ws, s);
+}
 
-    const bool decode = M <= kDecodeMaxM;
-    const int splits = decode ? gemv_splits(N, K) : 1;
-    QuantizeArgs q{};
-    q.X = x; q.M = M; q.K = K;
-    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
-    q.CA = at<int8_t>(ws, L.ca); q.SCA = at<float>(ws, L.sca);
-    q.outlier_idx = at<int32_t>(ws, L.idx); q.n_outliers = &hdr->n_outliers;
-    q.Xo = at<__half>(ws, L.xo); q.kcap = L.kcap;
-    q.W_outlier = static_cast<const __half *>(W_outlier); q.CB = CB; q.SCB = SCB; q.N = N;
-    if (!decode) q.Wo = at<__half>(ws, L.wo);
-    if (decode && splits > 1) {
-        q.acc = at<int32_t>(ws, L.acc); q.acc_words = N * 16;
-        q.cnt = at<uint32_t>(ws, L.cnt); q.cnt_words = ceil_div(N, 32);
-    }
-    if (cudaError_t e = launch_quantize(q, s)) return from_cuda(e);
+int int8lt_forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                            const void *W_outlier, float threshold, void *ws, size_t ws_bytes, void *stream) {
+    int st = check_forward_args(X, M, N, K, CB, SCB, W_outlier, threshold, nullptr, nullptr, true, false, ws,
+                                ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
+    return forward_quantize(X, M, N, K, CB, SCB, W_outlier, threshold, ws, static_cast<cudaStream_t>(stream));
+}
 
-    if (decode) {
-        GemvArgs g{};
-        g.CA = q.CA; g.CB = CB; g.SCA = q.SCA; g.SCB = SCB;
-        g.Xo = q.Xo; g.kcap = L.kcap; g.outlier_idx = q.outlier_idx; g.n_outliers = q.n_outliers;
-        g.W_outlier = q.W_outlier; g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
-        g.acc = q.acc; g.cnt = q.cnt;
-        g.M = M; g.N = N; g.K = K; g.splits = splits;
-        return from_cuda(launch_gemv(g, s));
-    }
-    GemmArgs g{};
-    g.CA = q.CA; g.CB = CB; g.SCA = q.SCA; g.SCB = SCB;
-    g.Xo = q.Xo; g.Wo = q.Wo; g.kcap = L.kcap; g.n_outliers = q.n_outliers;
-    g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
-    g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
-    return from_cuda(launch_gemm_tc(g, s));
+int int8lt_forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                          const void *W_outlier, const void *bias, void *Y, void *ws, size_t ws_bytes,
+                          void *stream) {
+    int st = check_forward_args(nullptr, M, N, K, CB, SCB, W_outlier, 0.f, bias, Y, false, true, ws, ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
+    return forward_matmul(M, N, K, CB, SCB, W_outlier, bias, Y, ws, static_cast<cudaStream_t>(stream));
 }
 
 int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K, int32_t *C,

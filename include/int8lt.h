@@ -143,6 +143,24 @@ int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K,
                    float threshold, const void *bias, void *Y,
                    void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * The two halves of int8lt_forward, for callers that want to time or
+ * schedule them apart; int8lt_forward is exactly _quantize then _matmul on
+ * the same stream and workspace, with identical arguments.
+ *   _quantize: outlier set O, CA/SCA and the fp16 outlier activations of X
+ *              into the workspace, plus (M > 16) the fp16 outlier weights
+ *              gathered from W_outlier (or CB/SCB).
+ *   _matmul  : the int8 GEMM (M > 16) or GEMV (M <= 16) with the fused
+ *              dequantization, outlier product and bias, writing Y. It reads
+ *              only what the preceding _quantize left in `ws`.
+ */
+int int8lt_forward_quantize(const void *X, int64_t M, int64_t N, int64_t K,
+                            const int8_t *CB, const float *SCB, const void *W_outlier,
+                            float threshold, void *ws, size_t ws_bytes, void *stream);
+int int8lt_forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                          const void *W_outlier, const void *bias, void *Y,
+                          void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- tests -- */
 
 /*

@@ -232,3 +232,17 @@ def test_validation_errors_raise():
     with pytest.raises(_lib.Int8ltError) as e:
         _lib.int8lt_forward(X, CB, SCB, W, 6.0, ws=ws)
     assert e.value.name == "INT8LT_ERR_WORKSPACE"
+
+
+def test_split_halves_equal_forward():
+    for w in (FCASES[1], FCASES[5]):
+        X, W, b = case_inputs(w)
+        Xd, Wd, bd = dev(X), dev(W), dev(b) if b is not None else None
+        CB, SCB = _lib.int8lt_prepare_weight(Wd)
+        y1 = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd)
+        ws = _lib.workspace(w.M, w.N, w.K)
+        y2 = torch.empty_like(y1)
+        _lib.int8lt_forward_quantize(Xd, CB, SCB, Wd, 6.0, ws)
+        _lib.int8lt_forward_matmul(w.M, CB, SCB, Wd, bd, y2, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
