@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libint8lt.so")
 STATUS = {
     0: "INT8LT_OK", 1: "INT8LT_ERR_NULL", 2: "INT8LT_ERR_SHAPE", 3: "INT8LT_ERR_ALIGN",
     4: "INT8LT_ERR_VALUE", 5: "INT8LT_ERR_WORKSPACE", 6: "INT8LT_ERR_CUDA",
-    7: "INT8LT_ERR_TIMEOUT", 8: "INT8LT_ERR_UNSUPPORTED",
+    7: "INT8LT_ERR_TIMEOUT", 8: "INT8LT_ERR_UNSUPPORTED", 9: "INT8LT_ERR_TOO_LARGE",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -27,7 +27,7 @@ EXPORTS = [
     "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
-    "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
+    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
 ]
 
 
@@ -53,6 +53,7 @@ _SIGS = {
     "int8lt_forward": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P, _SZ, _P]),
     "int8lt_forward_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _SZ, _P]),
     "int8lt_forward_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "int8lt_forward_static_scratch": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P]),
     "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
 }
@@ -208,6 +209,25 @@ def int8lt_forward_matmul(M: int, CB: torch.Tensor, SCB: torch.Tensor,
     _check("int8lt_forward_matmul",
            lib().int8lt_forward_matmul(M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier), _ptr(bias),
                                        _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
+def int8lt_forward_static_scratch(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                                  W_outlier: torch.Tensor | None, Y: torch.Tensor,
+                                  threshold: float = 6.0, bias: torch.Tensor | None = None,
+                                  stream=None) -> torch.Tensor:
+    """Decode-shape forward (M <= 16) whose scratch is the library's fixed device array.
+
+    For callers that cannot hand the layer a workspace: nothing is allocated by the call.
+    ``Y`` must be supplied (allocating it here would defeat the purpose). Calls that
+    overlap on the GPU share the one array and race; order them on one stream.
+    """
+    M, K = X.shape
+    N = CB.shape[0]
+    _check("int8lt_forward_static_scratch",
+           lib().int8lt_forward_static_scratch(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB),
+                                               _ptr(W_outlier), float(threshold), _ptr(bias),
+                                               _ptr(Y), _stream(stream)))
     return Y
 
 

@@ -119,6 +119,10 @@ int check_forward_args(const void *X, int64_t M, int64_t N, int64_t K, const int
     return check_device();
 }
 
+}  // namespace
+
+namespace int8lt {
+
 int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
                      const void *W_outlier, float threshold, void *ws, cudaStream_t s) {
     const WsLayout L = ws_layout(M, N, K);
@@ -168,7 +172,7 @@ int forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const floa
     return from_cuda(launch_gemm_tc(g, s));
 }
 
-}  // namespace
+}  // namespace int8lt
 
 extern "C" {
 
@@ -183,6 +187,8 @@ const char *int8lt_status_string(int status) {
         case INT8LT_ERR_CUDA: return "INT8LT_ERR_CUDA: a CUDA call or launch failed";
         case INT8LT_ERR_TIMEOUT: return "INT8LT_ERR_TIMEOUT: a kernel gave up a bounded wait";
         case INT8LT_ERR_UNSUPPORTED: return "INT8LT_ERR_UNSUPPORTED: device is not compute capability 10.0";
+        case INT8LT_ERR_TOO_LARGE:
+            return "INT8LT_ERR_TOO_LARGE: M > 16 or the call's scratch exceeds the 8 MiB static array";
         default: return "INT8LT_ERR_UNKNOWN";
     }
 }

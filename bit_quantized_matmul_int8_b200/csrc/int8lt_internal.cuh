@@ -119,6 +119,13 @@ cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s);
 
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 
+// The two halves of int8lt_forward on an already validated call; `ws` holds
+// at least ws_layout(M, N, K).total bytes. Return an int8lt_status.
+int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
+                     const void *W_outlier, float threshold, void *ws, cudaStream_t s);
+int forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB, const void *W_outlier,
+                   const void *bias, void *Y, void *ws, cudaStream_t s);
+
 // ------------------------------------------------------- device helpers --
 #ifdef __CUDACC__
 

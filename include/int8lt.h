@@ -61,7 +61,9 @@ typedef enum {
     INT8LT_ERR_WORKSPACE = 5,   /* ws_bytes < int8lt_workspace_size(...) */
     INT8LT_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
     INT8LT_ERR_TIMEOUT = 7,     /* a kernel gave up a bounded wait (device status) */
-    INT8LT_ERR_UNSUPPORTED = 8  /* current device is not compute capability 10.0 */
+    INT8LT_ERR_UNSUPPORTED = 8, /* current device is not compute capability 10.0 */
+    INT8LT_ERR_TOO_LARGE = 9    /* call exceeds the fixed scratch of
+                                   int8lt_forward_static_scratch */
 } int8lt_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -160,6 +162,31 @@ int int8lt_forward_quantize(const void *X, int64_t M, int64_t N, int64_t K,
 int int8lt_forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *SCB,
                           const void *W_outlier, const void *bias, void *Y,
                           void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Allocation-free forward for decode shapes. The paper has no counterpart:
+ * this is a deployment convenience of this library. It computes exactly what
+ * int8lt_forward computes (same kernels, same results) for M <= 16 tokens,
+ * but takes its scratch from a fixed 8 MiB array inside the library instead
+ * of a caller workspace, for callers that cannot allocate device memory: a
+ * plugin or engine that is handed only input and output buffers, a runtime
+ * whose device memory is owned by its own pool, or a decode loop that must
+ * not call cudaMalloc because it can synchronize the device.
+ *   - Limits: M <= 16, and the call's scratch (int8lt_workspace_size(M, N, K))
+ *     must fit the 8 MiB array (e.g. K = 12288 with N up to about 100k);
+ *     larger calls return INT8LT_ERR_TOO_LARGE without launching anything.
+ *   - The array lives on every GPU on which the library is loaded, until the
+ *     process exits. The first call on a device looks up the array's device
+ *     address (with that device current) and clears its header; make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the array. Each call re-initialises what
+ *     it reads, but calls whose kernels overlap on the GPU (unordered streams
+ *     or concurrent host threads) race on it and produce wrong results.
+ * Other arguments and errors as int8lt_forward.
+ */
+int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N, int64_t K,
+                                  const int8_t *CB, const float *SCB, const void *W_outlier,
+                                  float threshold, const void *bias, void *Y, void *stream);
 
 /* ---------------------------------------------------------------- tests -- */
 
