@@ -225,6 +225,23 @@ def run_reference(args, rank: int, world: int):
     emit(line, args.out)
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as tdist
+
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (max_ms * 1e-3)
+
+
 def emit(line: dict, out: str | None):
     s = json.dumps(line)
     print(s, flush=True)
@@ -316,21 +333,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize()
     if dist:
         tdist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     q_ms = [evq[s].elapsed_time(evm[s]) for s in range(K_steps)]
     m_ms = [evm[s].elapsed_time(eve[s]) for s in range(K_steps)]
-    if dist:
-        t = torch.tensor([elapsed_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     for ws in WSs:
         st = _lib.int8lt_read_device_status(ws)
         if st != 0:
             raise RuntimeError(f"device status {_lib.STATUS.get(st)} after the timed steps")
 
     ops = 2.0 * M * N * K
-    value = ops * K_steps * world / (elapsed_ms * 1e-3) / 1e12
-    tokens_per_s = M * K_steps * world / (elapsed_ms * 1e-3)
+    value = whole_job_rate(ops, K_steps, world, elapsed_ms) / 1e12
+    tokens_per_s = whole_job_rate(M, K_steps, world, elapsed_ms)
 
     # Roofline of the dominant kernel: the matmul half is one launch (GEMM or GEMV).
     m_avg = statistics.mean(m_ms) * 1e-3
@@ -380,14 +393,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         Yh.copy_(Yd, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": ops * n_e2e * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e = {"value": whole_job_rate(ops, n_e2e, world, e2e_ms) / 1e12, "unit": "TOPS",
            "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
-           "steps": n_e2e, "tokens_per_s": M * n_e2e * world / (e2e_ms * 1e-3)}
+           "steps": n_e2e, "tokens_per_s": whole_job_rate(M, n_e2e, world, e2e_ms)}
 
     if rank != 0:
         return
