@@ -11,7 +11,7 @@ namespace int8lt {
 
 int64_t flag_chunks_for(int64_t M, int64_t K) {
     const int64_t gx = ceil_div(K, kColsPerFlagCta);
-    int64_t c = ceil_div(2 * 148, gx);
+    int64_t c = ceil_div(4 * 148, gx);
     c = std::min<int64_t>(c, kMaxFlagChunks);
     c = std::min<int64_t>(c, ceil_div(std::max<int64_t>(M, 1), 32));
     return std::max<int64_t>(c, 1);

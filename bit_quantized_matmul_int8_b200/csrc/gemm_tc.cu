@@ -1,23 +1,33 @@
 // Prefill path of the LLM.int8() forward on sm_100a tensor cores.
 //
-// Computes, per 128 x 256 output tile,
+// Computes, per 256 x 256 output tile,
 //     Y = fp16( C * SCA[i] * SCB[j] / 127^2 + P + bias[j] )
 //     C = CA . CB^T    int8 x int8 -> int32   ("Int8 Matrix Multiplication with
 //                      16-bit Float Inputs and Outputs" and "Vector-wise
 //                      Quantization", LLM.int8() paper summary)
 //     P = Xo . Wo^T    fp16 x fp16 -> fp32    (the outlier columns, "The Core
 //                      of LLM.int8(): Mixed-precision Decomposition")
-// in one kernel:
-//   warp 0     TMA producer: 128-byte-swizzled K-major tiles of CA/CB (int8,
-//              128 wide) then Xo/Wo (fp16, 64 wide) into a 4-stage ring;
-//   warp 1     allocates tensor memory and issues tcgen05.mma (kind::i8 into
-//              TMEM columns [0,256), then kind::f16 into [256,512));
-//   warps 2-5  epilogue: tcgen05.ld both accumulators, dequantize in fp32,
-//              add P and bias, store fp16.
-// The outlier count |O| is read from device memory, so no host sync happens
-// between the quantize pass and this kernel. Every wait is bounded
-// (kWaitLimitNs); a wait that runs out sets the workspace status word and
-// the kernel winds down without touching Y.
+// in one persistent kernel run by CTA pairs (clusters of 2 SMs). Each tile
+// is computed by one pair with 2-SM tensor-core MMAs (tcgen05 cta_group::2):
+// each CTA stages its own 128 rows of A and its own half (128 rows) of B,
+// so per SM a 128 x 256 x 128 k-block needs 32 KB of operands instead of
+// 48 KB, and a 6-deep ring of stages fits in shared memory.
+//   warp 0     (both CTAs) TMA producer into a 6-stage ring; the loads of
+//              both CTAs complete on the leader CTA's full barrier;
+//   warp 1     (both CTAs) allocates the 512 tensor-memory columns; in the
+//              leader it issues the pair MMAs and multicasts the commits;
+//   warps 2-9  (both CTAs) epilogue on the CTA's 128 rows: tcgen05.ld the
+//              accumulator, dequantize in fp32, add P and bias, store fp16.
+// Outlier product, chosen on the device from |O| (no host sync):
+//   |O| <= kEpiOutlierMax: two int32 accumulators of 256 columns (double
+//       buffered: the epilogue of one tile overlaps the mainloop of the next)
+//       and P on the CUDA cores in the epilogue, from the row's Xo values in
+//       registers and the tile's Wo in shared memory; every fp16 x fp16
+//       product is exact in fp32, as on the tensor cores;
+//   |O| >  kEpiOutlierMax: one int32 accumulator (columns 0-255) and P as
+//       tcgen05 kind::f16 MMAs into an fp32 accumulator (columns 256-511).
+// Every wait is bounded (kWaitLimitNs); a wait that runs out sets the
+// workspace status word and the kernel winds down without touching Y.
 #include <algorithm>
 #include <mutex>
 
@@ -27,16 +37,22 @@ namespace int8lt {
 
 namespace {
 
-constexpr int BM = 128, BN = 256;
-constexpr int kStages = 4;
-constexpr int kStageA = BM * 128;  // bytes: 128 rows x 128 B
-constexpr int kStageB = BN * 128;  // bytes: 256 rows x 128 B
-constexpr int kThreads = 192;
+constexpr int BM = 256, BN = 256;         // pair tile
+constexpr int kCtaRows = 128;             // rows of A (and of B) staged per CTA
+constexpr int kStages = 6;
+constexpr int kStageA = kCtaRows * 128;   // bytes: 128 rows x 128 B
+constexpr int kStageB = kCtaRows * 128;   // bytes: 128 rows x 128 B (half of N)
+constexpr uint32_t kTxBytes = 2 * (kStageA + kStageB);  // both CTAs, counted by the leader
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccOutlierCol = 256;
+constexpr int kEpiOutlierMax = 32;
+constexpr int kEpiBarrier = 1;            // named barrier of the epilogue warps
+constexpr uint16_t kPairMask = 0x3;       // both CTAs of the cluster
 
 // Instruction descriptors (tcgen05 .kind::i8 / .kind::f16): dense, K-major
-// A and B, N = 256 (bits 17-22 hold N/8), M = 128 (bits 24-28 hold M/16).
+// A and B, N = 256 (bits 17-22 hold N/8), M = 256 (bits 24-28 hold M/16).
 constexpr uint32_t kIdescI8 = (2u << 4)      // D = s32
                               | (1u << 7)    // A = signed int8
                               | (1u << 10)   // B = signed int8
@@ -44,36 +60,53 @@ constexpr uint32_t kIdescI8 = (2u << 4)      // D = s32
 constexpr uint32_t kIdescF16 = (1u << 4)     // D = f32, A = B = f16 (0)
                                | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-constexpr size_t kSmemTiles = (size_t)kStages * (kStageA + kStageB);
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kSmemTiles + 256 /*barriers*/ + 2 * BN * 4;
-
 struct __align__(8) Ctrl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t acc;
+    uint64_t full[kStages];     // leader: both CTAs' stage bytes landed
+    uint64_t empty[kStages];    // each CTA: the pair MMAs are done with the stage
+    uint64_t acc_full[2];       // each CTA: the accumulator buffer is complete
+    uint64_t acc_empty[2];      // leader: both CTAs' epilogues have read the buffer
+    uint64_t drain;             // each CTA: every pair MMA has finished
     uint32_t tmem_base;
     uint32_t abort;
+    uint32_t epi_abort[2];      // epilogue votes, one slot per tile parity
 };
+
+constexpr size_t kSmemTiles = (size_t)kStages * (kStageA + kStageB);
+constexpr size_t kOffCtrl = kSmemTiles;
+constexpr size_t kOffScb = kOffCtrl + 256;
+constexpr size_t kOffBias = kOffScb + BN * 4;
+constexpr size_t kOffWo = kOffBias + BN * 4;                     // fp16 [kEpiOutlierMax][BN]
+constexpr size_t kSmemUsed = kOffWo + (size_t)kEpiOutlierMax * BN * 2;
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kSmemUsed;
+static_assert(sizeof(Ctrl) <= 256, "control block");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync %0, %1;" ::"r"(kEpiBarrier), "r"(kEpiThreads) : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
-               const GemmArgs a, const int num_m_tiles) {
+               const GemmArgs a, const int num_m_tiles, const int num_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * kStageA;
-    Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem + kSmemTiles);
-    float *s_scb = reinterpret_cast<float *>(smem + kSmemTiles + 256);
-    float *s_bias = s_scb + BN;
+    Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem + kOffCtrl);
+    float *s_scb = reinterpret_cast<float *>(smem + kOffScb);
+    float *s_bias = reinterpret_cast<float *>(smem + kOffBias);
+    __half *s_wo = reinterpret_cast<__half *>(smem + kOffWo);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x % num_m_tiles, nt = blockIdx.x / num_m_tiles;
-    const int64_t m0 = (int64_t)mt * BM, n0 = (int64_t)nt * BN;
+    const uint32_t rank = cluster_ctarank();          // 0: leader, 1: follower
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int nkb = (int)ceil_div(a.K, 128);
     const int n_out = a.n_outliers ? *a.n_outliers : 0;
-    const int n_mma_o = (n_out + 15) >> 4;   // fp16 MMAs of K = 16
-    const int nkb_o = (n_out + 63) >> 6;     // fp16 k-blocks of 64
+    const bool mma_out = n_out > kEpiOutlierMax;       // outlier product on the tensor cores
+    const int nbuf = mma_out ? 1 : 2;                  // accumulator buffers in TMEM
+    const int n_mma_o = mma_out ? (n_out + 15) >> 4 : 0;   // fp16 MMAs of K = 16
+    const int nkb_o = mma_out ? (n_out + 63) >> 6 : 0;     // fp16 k-blocks of 64
     const int total_kb = nkb + nkb_o;
 
     if (threadIdx.x == 0) {
@@ -81,32 +114,31 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             mbar_init(smem_u32(&ctrl->full[s]), 1);
             mbar_init(smem_u32(&ctrl->empty[s]), 1);
         }
-        mbar_init(smem_u32(&ctrl->acc), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&ctrl->acc_full[b]), 1);
+            mbar_init(smem_u32(&ctrl->acc_empty[b]), 2 * kEpiWarps);
+        }
+        mbar_init(smem_u32(&ctrl->drain), 1);
         ctrl->abort = 0;
+        ctrl->epi_abort[0] = ctrl->epi_abort[1] = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
     if (threadIdx.x == 32) {
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
-        if (nkb_o) {
+        if (mma_out) {
             tma_prefetch(&tmXo);
             tma_prefetch(&tmWo);
         }
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&ctrl->tmem_base), kTmemCols);
-        tmem_relinquish();
-    }
-    if (warp >= 2) {
-        for (int c = threadIdx.x - 64; c < BN; c += 128) {
-            const int64_t j = n0 + c;
-            s_scb[c] = (a.SCB && j < a.N) ? a.SCB[j] : 0.f;
-            s_bias[c] = (a.bias && j < a.N) ? __half2float(a.bias[j]) : 0.f;
-        }
+        tmem_alloc_pair(smem_u32(&ctrl->tmem_base), kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
     volatile uint32_t *abort_flag = &ctrl->abort;
@@ -117,85 +149,163 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
-            for (int kb = 0; kb < total_kb; ++kb) {
-                if (*abort_flag) break;
-                if (!mbar_wait_bounded(smem_u32(&ctrl->empty[stage]), phase ^ 1u, kWaitLimitNs)) {
-                    *abort_flag = 1;
-                    record_timeout(a.status);
-                    break;
+            for (int tile = pair; tile < num_tiles && !*abort_flag; tile += num_pairs) {
+                const int32_t m0 = (tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
+                const int32_t n0 = (tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    if (*abort_flag) break;
+                    if (!mbar_wait_bounded(smem_u32(&ctrl->empty[stage]), phase ^ 1u, kWaitLimitNs)) {
+                        *abort_flag = 1;
+                        record_timeout(a.status);
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&ctrl->full[stage]);
+                    if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
+                    const uint32_t fb_leader = mapa_shared(fb, 0);
+                    if (kb < nkb) {
+                        tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmA, fb_leader, kb * 128, m0);
+                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmB, fb_leader, kb * 128, n0);
+                    } else {
+                        const int ko = (kb - nkb) * 64;
+                        tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmXo, fb_leader, ko, m0);
+                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmWo, fb_leader, ko, n0);
+                    }
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
-                const uint32_t fb = smem_u32(&ctrl->full[stage]);
-                mbar_arrive_expect_tx(fb, kStageA + kStageB);
-                if (kb < nkb) {
-                    tma_load_2d(smem_u32(sA + stage * kStageA), &tmA, fb, kb * 128, (int32_t)m0);
-                    tma_load_2d(smem_u32(sB + stage * kStageB), &tmB, fb, kb * 128, (int32_t)n0);
-                } else {
-                    const int ko = (kb - nkb) * 64;
-                    tma_load_2d(smem_u32(sA + stage * kStageA), &tmXo, fb, ko, (int32_t)m0);
-                    tma_load_2d(smem_u32(sB + stage * kStageB), &tmWo, fb, ko, (int32_t)n0);
-                }
-                ++issued;
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
             }
-            // Do not leave while copies this thread started are in flight.
+            // Do not leave while copies this thread started are in flight:
+            // a stage is free again once the pair MMAs have consumed it.
             for (int u = max(0, issued - kStages); u < issued; ++u) {
                 const int s = u % kStages;
-                if (!mbar_wait_bounded(smem_u32(&ctrl->full[s]), (uint32_t)((u / kStages) & 1), kWaitLimitNs)) {
+                if (!mbar_wait_bounded(smem_u32(&ctrl->empty[s]), (uint32_t)((u / kStages) & 1), kWaitLimitNs)) {
                     record_timeout(a.status);
                     break;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer --
+        if (lane == 0 && rank == 0) {
+            // ----------------------------------------- MMA issuer (leader) --
             int stage = 0;
             uint32_t phase = 0;
-            for (int kb = 0; kb < total_kb; ++kb) {
-                if (*abort_flag) break;
-                if (!mbar_wait_bounded(smem_u32(&ctrl->full[stage]), phase, kWaitLimitNs)) {
+            int it = 0;  // local tile count
+            for (int tile = pair; tile < num_tiles && !*abort_flag; tile += num_pairs, ++it) {
+                const int buf = it % nbuf;
+                const uint32_t use = (uint32_t)(it / nbuf);
+                if (!mbar_wait_bounded(smem_u32(&ctrl->acc_empty[buf]), (use & 1u) ^ 1u, kWaitLimitNs)) {
                     *abort_flag = 1;
                     record_timeout(a.status);
                     break;
                 }
                 tc_fence_after();
-                const uint64_t da = sdesc_k_sw128(smem_u32(sA + stage * kStageA));
-                const uint64_t db = sdesc_k_sw128(smem_u32(sB + stage * kStageB));
-                if (kb < nkb) {
+                const uint32_t d_i32 = tmem + (uint32_t)(buf * 256);
+                const uint32_t d_f32 = tmem + 256;
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    if (*abort_flag) break;
+                    if (!mbar_wait_bounded(smem_u32(&ctrl->full[stage]), phase, kWaitLimitNs)) {
+                        *abort_flag = 1;
+                        record_timeout(a.status);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sdesc_k_sw128(smem_u32(sA + stage * kStageA));
+                    const uint64_t db = sdesc_k_sw128(smem_u32(sB + stage * kStageB));
+                    if (kb < nkb) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 4 x (K = 32 int8 = 32 bytes)
-                        mma_i8(tmem, da + 2 * k, db + 2 * k, kIdescI8, (kb | k) != 0);
-                } else {
-                    const int kbo = kb - nkb;
-                    const int nk = min(4, n_mma_o - kbo * 4);
-                    for (int k = 0; k < nk; ++k)  // K = 16 fp16 = 32 bytes each
-                        mma_f16(tmem + kAccOutlierCol, da + 2 * k, db + 2 * k, kIdescF16, (kbo | k) != 0);
+                        for (int k = 0; k < 4; ++k)  // 4 x (K = 32 int8 = 32 bytes)
+                            mma_i8_pair(d_i32, da + 2 * k, db + 2 * k, kIdescI8, (kb | k) != 0);
+                    } else {
+                        const int kbo = kb - nkb;
+                        const int nk = min(4, n_mma_o - kbo * 4);
+                        for (int k = 0; k < nk; ++k)  // K = 16 fp16 = 32 bytes each
+                            mma_f16_pair(d_f32, da + 2 * k, db + 2 * k, kIdescF16, (kbo | k) != 0);
+                    }
+                    mma_commit_pair(smem_u32(&ctrl->empty[stage]), kPairMask);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
-                mma_commit(smem_u32(&ctrl->empty[stage]));
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                // lands in both CTAs when this tile's MMAs are done
+                mma_commit_pair(smem_u32(&ctrl->acc_full[buf]), kPairMask);
             }
-            // Always signal the epilogue; the arrive lands once every MMA
-            // issued above has finished, so TMEM is safe to read (or free).
-            mma_commit(smem_u32(&ctrl->acc));
-            if (!mbar_wait_bounded(smem_u32(&ctrl->acc), 0, kWaitLimitNs)) record_timeout(a.status);
+            // Nothing may still write either CTA's TMEM when it is freed.
+            mma_commit_pair(smem_u32(&ctrl->drain), kPairMask);
+        }
+        if (lane == 0) {
+            if (!mbar_wait_bounded(smem_u32(&ctrl->drain), 0, kWaitLimitNs)) record_timeout(a.status);
         }
     } else {
         // ---------------------------------------------------- epilogue --
-        const int q = warp & 3;  // this warp may touch TMEM lanes [32q, 32q + 32)
-        const int64_t row = m0 + q * 32 + lane;
-        bool ok = mbar_wait_bounded(smem_u32(&ctrl->acc), 0, kWaitLimitNs);
-        if (!ok) record_timeout(a.status);
-        ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
-        tc_fence_after();
-        if (ok) {
+        const int ew = warp - 2;                 // 0..7
+        const int q = warp & 3;                  // TMEM lanes [32q, 32q + 32) are this warp's
+        const int hcol = ew >> 2;                // columns [128 hcol, 128 hcol + 128)
+        const int et = threadIdx.x - 64;         // 0..255
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const bool cuda_out = !mma_out && n_out > 0;
+        int it = 0;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
+            const int64_t m0 = (int64_t)(tile % num_m_tiles) * BM + rank * kCtaRows;
+            const int64_t n0 = (int64_t)(tile / num_m_tiles) * BN;
+            const int buf = it % nbuf;
+            const uint32_t use = (uint32_t)(it / nbuf);
+            // Wait for the accumulator, then decide together whether to go
+            // on: every epilogue warp votes before the barrier and reads the
+            // same slot after it, so all of them leave the loop together.
+            bool ok = mbar_wait_bounded(smem_u32(&ctrl->acc_full[buf]), use & 1u, kWaitLimitNs);
+            if (!ok) record_timeout(a.status);
+            ok = __all_sync(0xffffffffu, ok);
+            volatile uint32_t *vote = &ctrl->epi_abort[it & 1];
+            if (lane == 0 && (!ok || *abort_flag)) *vote = 1;
+            // Stage this tile's column data (the previous tile's readers are done).
+            epi_sync();
+            if (*vote) {
+                *abort_flag = 1;
+                break;
+            }
+            if (!a.C32) {
+                for (int c = et; c < BN; c += kEpiThreads) {
+                    const int64_t j = n0 + c;
+                    s_scb[c] = j < a.N ? a.SCB[j] : 0.f;
+                    s_bias[c] = (a.bias && j < a.N) ? __half2float(a.bias[j]) : 0.f;
+                }
+                if (cuda_out) {
+                    const int n16 = (n_out + 15) & ~15;
+                    for (int i = et; i < n16 * BN; i += kEpiThreads) {
+                        const int t = i / BN, c = i % BN;
+                        const int64_t j = n0 + c;
+                        s_wo[t * BN + c] = j < a.N ? a.Wo[j * a.kcap + t] : __float2half_rn(0.f);
+                    }
+                }
+            }
+            epi_sync();
+            tc_fence_after();
+            const int64_t row = m0 + q * 32 + lane;
             const bool row_ok = row < a.M;
             const float rs = (row_ok && a.SCA) ? a.SCA[row] * (1.0f / 16129.0f) : 0.f;
-            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-            for (int c = 0; c < BN; c += 32) {
+            // This row's outlier activations (CUDA-core outlier product).
+            __half2 xo2[kEpiOutlierMax / 2];
+            if (cuda_out) {
+#pragma unroll
+                for (int t = 0; t < kEpiOutlierMax / 2; ++t)
+                    xo2[t] = (row_ok && 2 * t < n_out)
+                                 ? *reinterpret_cast<const __half2 *>(a.Xo + row * a.kcap + 2 * t)
+                                 : __floats2half2_rn(0.f, 0.f);
+            }
+            const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
+            for (int cc = 0; cc < 128; cc += 32) {
+                const int c = hcol * 128 + cc;  // column within the tile
                 uint32_t acc[32], po[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + c, acc);
-                if (n_out > 0) tmem_ld_32x32b_x32(tmem + lane_base + kAccOutlierCol + c, po);
+                tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+                if (mma_out) tmem_ld_32x32b_x32(tmem + lane_base + 256 + col0 + cc, po);
                 tmem_ld_wait();
+                if (cc == 96) {
+                    // Every TMEM read of this buffer is done: hand it back to
+                    // the leader's MMA warp.
+                    tc_fence_before();
+                    if (lane == 0) {
+                        const uint32_t eb = smem_u32(&ctrl->acc_empty[buf]);
+                        if (rank == 0) mbar_arrive(eb); else mbar_arrive_cluster(mapa_shared(eb, 0));
+                    }
+                }
                 if (!row_ok || n0 + c >= a.N) continue;
                 if (a.C32) {
                     int32_t *dst = a.C32 + row * a.N + n0 + c;
@@ -206,16 +316,37 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                 make_int4((int)acc[4 * v], (int)acc[4 * v + 1], (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
                     continue;
                 }
+                float y[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    y[j] = (float)(int32_t)acc[j] * (rs * s_scb[c + j]) + s_bias[c + j];
+                    if (mma_out) y[j] += __uint_as_float(po[j]);
+                }
+                if (cuda_out) {
+                    for (int t2 = 0; 2 * t2 < n_out; ++t2) {
+                        const float2 xf = __half22float2(xo2[t2]);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const float xv = h ? xf.y : xf.x;
+                            const uint4 *w4 = reinterpret_cast<const uint4 *>(s_wo + (2 * t2 + h) * BN + c);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                const uint4 wv = w4[v];
+                                const __half2 *wh = reinterpret_cast<const __half2 *>(&wv);
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const float2 wf = __half22float2(wh[u]);
+                                    y[8 * v + 2 * u] = fmaf(xv, wf.x, y[8 * v + 2 * u]);
+                                    y[8 * v + 2 * u + 1] = fmaf(xv, wf.y, y[8 * v + 2 * u + 1]);
+                                }
+                            }
+                        }
+                    }
+                }
                 uint32_t packed[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                    float y0 = (float)(int32_t)acc[j] * (rs * s_scb[c + j]) + s_bias[c + j];
-                    float y1 = (float)(int32_t)acc[j + 1] * (rs * s_scb[c + j + 1]) + s_bias[c + j + 1];
-                    if (n_out > 0) {
-                        y0 += __uint_as_float(po[j]);
-                        y1 += __uint_as_float(po[j + 1]);
-                    }
-                    __half2 h = __floats2half2_rn(y0, y1);
+                    __half2 h = __floats2half2_rn(y[j], y[j + 1]);
                     packed[j >> 1] = *reinterpret_cast<uint32_t *>(&h);
                 }
                 __half *dst = a.Y + row * a.N + n0 + c;
@@ -228,11 +359,14 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     }
 
+    // Teardown: the pair's peer must be done signalling this CTA's barriers
+    // and its MMAs done with this CTA's TMEM before TMEM is freed and the CTA exits.
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -273,16 +407,18 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int g_num_sms[64];  // resident CTA pairs per device
+
 }  // namespace
 
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     CUtensorMap mA, mB, mXo, mWo;
-    if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CA, a.K, a.M, a.K, 128, BM) ||
-        !make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CB, a.K, a.N, a.K, 128, BN))
+    if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CA, a.K, a.M, a.K, 128, kCtaRows) ||
+        !make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CB, a.K, a.N, a.K, 128, kCtaRows))
         return cudaErrorInvalidValue;
     if (a.Xo && a.Wo && a.n_outliers) {
-        if (!make_map(&mXo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Xo, a.kcap, a.M, a.kcap * 2, 64, BM) ||
-            !make_map(&mWo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Wo, a.kcap, a.N, a.kcap * 2, 64, BN))
+        if (!make_map(&mXo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Xo, a.kcap, a.M, a.kcap * 2, 64, kCtaRows) ||
+            !make_map(&mWo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Wo, a.kcap, a.N, a.kcap * 2, 64, kCtaRows))
             return cudaErrorInvalidValue;
     } else {
         mXo = mA;  // never read: |O| = 0 without outlier buffers
@@ -293,14 +429,33 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     cudaError_t attr_err = cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;  // CTA pairs
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     std::call_once(attr_once[dev & 63], [&] {
         attr_err = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (attr_err != cudaSuccess) return;
+        // How many CTA pairs can be resident at once (a pair needs two SMs of one GPC).
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3(2, 1, 1);
+        int clusters = 0;
+        attr_err = cudaOccupancyMaxActiveClusters(&clusters, (void *)gemm_i8_kernel, &q);
+        g_num_sms[dev & 63] = clusters;
     });
     if (attr_err != cudaSuccess) return attr_err;
     const int num_m_tiles = (int)ceil_div(a.M, BM);
     const int64_t tiles = (int64_t)num_m_tiles * ceil_div(a.N, BN);
-    gemm_i8_kernel<<<(unsigned)tiles, kThreads, kSmemBytes, s>>>(mA, mB, mXo, mWo, a, num_m_tiles);
-    return cudaGetLastError();
+    const int pairs = g_num_sms[dev & 63] > 0 ? g_num_sms[dev & 63] : 74;
+    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(tiles, pairs), 1, 1);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, a, num_m_tiles, (int)tiles);
 }
 
 }  // namespace int8lt
