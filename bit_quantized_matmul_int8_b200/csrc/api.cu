@@ -9,14 +9,6 @@
 
 namespace int8lt {
 
-int64_t flag_chunks_for(int64_t M, int64_t K) {
-    const int64_t gx = ceil_div(K, kColsPerFlagCta);
-    int64_t c = ceil_div(4 * 148, gx);
-    c = std::min<int64_t>(c, kMaxFlagChunks);
-    c = std::min<int64_t>(c, ceil_div(std::max<int64_t>(M, 1), 32));
-    return std::max<int64_t>(c, 1);
-}
-
 static size_t align_up(size_t v) { return (v + 1023) & ~size_t(1023); }
 
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
@@ -24,10 +16,9 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
     L.M = M; L.N = N; L.K = K;
     L.kwords = ceil_div(K, 32);
     L.kcap = round_up(K, 64);
-    L.flag_chunks = flag_chunks_for(M, K);
     size_t off = 0;
-    L.hdr = off;   off += align_up(sizeof(WsHeader));
-    L.flags = off; off += align_up((size_t)L.flag_chunks * L.kwords * 4);
+    L.hdr = off;     off += align_up(sizeof(WsHeader));
+    L.bitmaps = off; off += align_up(kWsInitBytes - kWsBitmapOffset);
     L.idx = off;   off += align_up((size_t)K * 4);
     L.sca = off;   off += align_up((size_t)M * 4);
     L.ca = off;    off += align_up((size_t)M * K);
@@ -128,14 +119,11 @@ int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_
     const WsLayout L = ws_layout(M, N, K);
     const __half *x = static_cast<const __half *>(X);
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
-    const uint16_t tb = threshold_bits(threshold);
-    uint32_t *flags = at<uint32_t>(ws, L.flags);
-    if (cudaError_t e = launch_outlier_flags(x, M, K, tb, flags, L.flag_chunks, s)) return from_cuda(e);
     const bool decode = M <= kDecodeMaxM;
     const int splits = decode ? gemv_splits(N, K) : 1;
     QuantizeArgs q{};
     q.X = x; q.M = M; q.K = K;
-    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
+    q.hdr = hdr; q.bitmaps = at<uint32_t>(ws, L.bitmaps); q.tbits = threshold_bits(threshold);
     q.CA = at<int8_t>(ws, L.ca); q.SCA = at<float>(ws, L.sca);
     q.outlier_idx = at<int32_t>(ws, L.idx); q.n_outliers = &hdr->n_outliers;
     q.Xo = at<__half>(ws, L.xo); q.kcap = L.kcap;
@@ -204,7 +192,9 @@ int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream) {
     if (!ws) return INT8LT_ERR_NULL;
     if (ws_bytes < sizeof(WsHeader)) return INT8LT_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return INT8LT_ERR_ALIGN;
-    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+    // header (status, outlier count, quantize generation and barrier count)
+    // and both column bitmaps
+    return from_cuda(cudaMemsetAsync(ws, 0, std::min(ws_bytes, kWsInitBytes), static_cast<cudaStream_t>(stream)));
 }
 
 int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream) {
@@ -248,14 +238,11 @@ int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold, i
     }
     if (int st = check_device()) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const uint16_t tb = threshold_bits(threshold);
-    uint32_t *flags = at<uint32_t>(ws, L.flags);
-    if (cudaError_t e = launch_outlier_flags(static_cast<const __half *>(X), M, K, tb, flags, L.flag_chunks, s))
-        return from_cuda(e);
     QuantizeArgs q{};
     q.X = static_cast<const __half *>(X);
     q.M = M; q.K = K;
-    q.flags = flags; q.flag_chunks = L.flag_chunks; q.tbits = tb;
+    q.hdr = at<WsHeader>(ws, L.hdr); q.bitmaps = at<uint32_t>(ws, L.bitmaps);
+    q.tbits = threshold_bits(threshold);
     q.CA = CA; q.SCA = SCA; q.outlier_idx = outlier_idx; q.n_outliers = n_outliers;
     q.kcap = L.kcap;
     return from_cuda(launch_quantize(q, s));

@@ -17,7 +17,9 @@
 //   warp 1     (both CTAs) allocates the 512 tensor-memory columns; in the
 //              leader it issues the pair MMAs and multicasts the commits;
 //   warps 2-9  (both CTAs) epilogue on the CTA's 128 rows: tcgen05.ld the
-//              accumulator, dequantize in fp32, add P and bias, store fp16.
+//              accumulator, dequantize in fp32, add P and bias, and store fp16
+//              through shared memory with TMA (32 x 32 boxes, double buffered
+//              per warp), so the epilogue warps never wait on global stores.
 // Outlier product, chosen on the device from |O| (no host sync):
 //   |O| <= kEpiOutlierMax: two int32 accumulators of 256 columns (double
 //       buffered: the epilogue of one tile overlaps the mainloop of the next)
@@ -39,7 +41,7 @@ namespace {
 
 constexpr int BM = 256, BN = 256;         // pair tile
 constexpr int kCtaRows = 128;             // rows of A (and of B) staged per CTA
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 constexpr int kStageA = kCtaRows * 128;   // bytes: 128 rows x 128 B
 constexpr int kStageB = kCtaRows * 128;   // bytes: 128 rows x 128 B (half of N)
 constexpr uint32_t kTxBytes = 2 * (kStageA + kStageB);  // both CTAs, counted by the leader
@@ -71,8 +73,11 @@ struct __align__(8) Ctrl {
     uint32_t epi_abort[2];      // epilogue votes, one slot per tile parity
 };
 
+constexpr int kStoreBox = 32;                                    // Y staged in 32 x 32 fp16 boxes
+constexpr size_t kStoreBufBytes = kStoreBox * kStoreBox * 2;     // 2 KB
 constexpr size_t kSmemTiles = (size_t)kStages * (kStageA + kStageB);
-constexpr size_t kOffCtrl = kSmemTiles;
+constexpr size_t kOffStage = kSmemTiles;                         // [kEpiWarps][2] store boxes
+constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * 2 * kStoreBufBytes;
 constexpr size_t kOffScb = kOffCtrl + 256;
 constexpr size_t kOffBias = kOffScb + BN * 4;
 constexpr size_t kOffWo = kOffBias + BN * 4;                     // fp16 [kEpiOutlierMax][BN]
@@ -88,7 +93,8 @@ __device__ __forceinline__ void epi_sync() {
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
-               const GemmArgs a, const int num_m_tiles, const int num_tiles) {
+               const __grid_constant__ CUtensorMap tmY, const GemmArgs a, const int num_m_tiles,
+               const int num_tiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -97,6 +103,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     float *s_scb = reinterpret_cast<float *>(smem + kOffScb);
     float *s_bias = reinterpret_cast<float *>(smem + kOffBias);
     __half *s_wo = reinterpret_cast<__half *>(smem + kOffWo);
+    uint8_t *s_stage = smem + kOffStage;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();          // 0: leader, 1: follower
@@ -127,6 +134,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (threadIdx.x == 32) {
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
+        if (!a.C32) tma_prefetch(&tmY);
         if (mma_out) {
             tma_prefetch(&tmXo);
             tma_prefetch(&tmWo);
@@ -241,6 +249,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int et = threadIdx.x - 64;         // 0..255
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const bool cuda_out = !mma_out && n_out > 0;
+        int sbuf = 0;  // which of the warp's two store boxes is next
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
             const int64_t m0 = (int64_t)(tile % num_m_tiles) * BM + rank * kCtaRows;
@@ -306,8 +315,9 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         if (rank == 0) mbar_arrive(eb); else mbar_arrive_cluster(mapa_shared(eb, 0));
                     }
                 }
-                if (!row_ok || n0 + c >= a.N) continue;
+                if (n0 + c >= a.N) continue;  // whole chunk past the last column
                 if (a.C32) {
+                    if (!row_ok) continue;
                     int32_t *dst = a.C32 + row * a.N + n0 + c;
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
@@ -317,13 +327,24 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     continue;
                 }
                 float y[32];
+                const float4 *sc4 = reinterpret_cast<const float4 *>(s_scb + c);
+                const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias + c);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    y[j] = (float)(int32_t)acc[j] * (rs * s_scb[c + j]) + s_bias[c + j];
-                    if (mma_out) y[j] += __uint_as_float(po[j]);
+                for (int v = 0; v < 8; ++v) {
+                    const float4 sc = sc4[v], bi = bi4[v];
+                    y[4 * v + 0] = fmaf((float)(int32_t)acc[4 * v + 0] * rs, sc.x, bi.x);
+                    y[4 * v + 1] = fmaf((float)(int32_t)acc[4 * v + 1] * rs, sc.y, bi.y);
+                    y[4 * v + 2] = fmaf((float)(int32_t)acc[4 * v + 2] * rs, sc.z, bi.z);
+                    y[4 * v + 3] = fmaf((float)(int32_t)acc[4 * v + 3] * rs, sc.w, bi.w);
+                }
+                if (mma_out) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(po[j]);
                 }
                 if (cuda_out) {
-                    for (int t2 = 0; 2 * t2 < n_out; ++t2) {
+#pragma unroll
+                    for (int t2 = 0; t2 < kEpiOutlierMax / 2; ++t2) {
+                        if (2 * t2 >= n_out) break;  // uniform across the CTA
                         const float2 xf = __half22float2(xo2[t2]);
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
@@ -349,14 +370,27 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     __half2 h = __floats2half2_rn(y[j], y[j + 1]);
                     packed[j >> 1] = *reinterpret_cast<uint32_t *>(&h);
                 }
-                __half *dst = a.Y + row * a.N + n0 + c;
+                // Stage the warp's 32 x 32 box in shared memory (64-byte swizzle:
+                // 16-byte chunk i of row r sits at chunk i ^ ((r >> 1) & 3), which
+                // keeps the four stores of each row conflict-free) and hand it to
+                // the TMA engine. Rows and columns past M and N are clipped by it.
+                if (lane == 0) bulk_wait_read_1();  // this buffer's previous store has read it
+                __syncwarp();
+                uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    if (n0 + c + 8 * v < a.N)
-                        reinterpret_cast<uint4 *>(dst)[v] =
-                            make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
+                        make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, smem_u32(box), (int32_t)(n0 + c), (int32_t)(m0 + q * 32));
+                    bulk_commit_group();
+                }
+                sbuf ^= 1;
             }
         }
+        if (lane == 0) bulk_wait_all();  // every store of this warp has finished
     }
 
     // Teardown: the pair's peer must be done signalling this CTA's barriers
@@ -395,7 +429,8 @@ EncodeTiledFn get_encode_fn() {
 // row pitch `pitch_bytes`; box of box_inner x box_outer; 128-byte swizzle;
 // out-of-range elements read as zero.
 bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -403,7 +438,7 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -424,6 +459,10 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
         mXo = mA;  // never read: |O| = 0 without outlier buffers
         mWo = mB;
     }
+    CUtensorMap mY = mA;  // never read when the raw int32 sums are stored instead
+    if (!a.C32 && !make_map(&mY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Y, a.N, a.M, a.N * 2, kStoreBox, kStoreBox,
+                            CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
     static std::once_flag attr_once[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -455,7 +494,7 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     const int64_t tiles = (int64_t)num_m_tiles * ceil_div(a.N, BN);
     const int pairs = g_num_sms[dev & 63] > 0 ? g_num_sms[dev & 63] : 74;
     cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(tiles, pairs), 1, 1);
-    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, a, num_m_tiles, (int)tiles);
+    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, mY, a, num_m_tiles, (int)tiles);
 }
 
 }  // namespace int8lt

@@ -13,8 +13,7 @@ namespace int8lt {
 
 constexpr int64_t kMaxK = 133144;       // 127^2 * K < 2^31
 constexpr int kDecodeMaxM = 16;         // M <= 16 takes the GEMV path
-constexpr int kColsPerFlagCta = 64;     // phase-A column strip: 8 lanes x 8 fp16 = 128 bytes
-constexpr int kMaxFlagChunks = 8;       // row chunks of phase A (partial bitmaps)
+constexpr int64_t kMaxKwords = (kMaxK + 31) / 32;  // words of the largest column bitmap
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every in-kernel wait
 
 // Device status bits (workspace header word 0).
@@ -24,22 +23,26 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 __host__ __device__ __forceinline__ int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
 // Byte offsets of the workspace sections (every section 1024-byte aligned).
+// The header and the two column bitmaps sit at fixed offsets whatever the
+// shape, so one zeroing of the first kWsInitBytes prepares any workspace.
 struct WsLayout {
     int64_t M, N, K;
     int64_t kwords;        // ceil(K / 32): words of one column bitmap
     int64_t kcap;          // round_up(K, 64): row pitch (elements) of Xo / Wo
-    int64_t flag_chunks;   // phase-A row chunks actually used
-    size_t hdr, flags, idx, sca, ca, xo, wo, acc, cnt, total;
+    size_t hdr, bitmaps, idx, sca, ca, xo, wo, acc, cnt, total;
 };
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K);
-int64_t flag_chunks_for(int64_t M, int64_t K);
 
 // Workspace header (first 256 bytes).
 struct WsHeader {
     uint32_t status;       // kStatus* bits, sticky until read
     int32_t n_outliers;    // |O| of the last quantize pass
-    uint32_t pad[62];
+    uint32_t qgen;         // quantize launches so far: selects this launch's bitmap
+    uint32_t bar_count;    // arrivals at the quantize grid barrier (0 between launches)
+    uint32_t pad[60];
 };
+constexpr size_t kWsBitmapOffset = 1024;
+constexpr size_t kWsInitBytes = kWsBitmapOffset + 2 * (size_t)kMaxKwords * 4;
 
 // ------------------------------------------------------------- launchers --
 
@@ -49,15 +52,11 @@ uint16_t threshold_bits(float threshold);
 cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
                                   cudaStream_t s);
 
-// Phase A: partial column-outlier bitmaps [flag_chunks][kwords].
-cudaError_t launch_outlier_flags(const __half *X, int64_t M, int64_t K, uint16_t tbits,
-                                 uint32_t *flags, int64_t flag_chunks, cudaStream_t s);
-
 struct QuantizeArgs {
     const __half *X;
     int64_t M, K;
-    const uint32_t *flags;
-    int64_t flag_chunks;
+    WsHeader *hdr;            // generation counter and grid-barrier count
+    uint32_t *bitmaps;        // 2 x kMaxKwords words, one per launch parity
     uint16_t tbits;
     int8_t *CA;
     float *SCA;
@@ -77,6 +76,8 @@ struct QuantizeArgs {
     uint32_t *cnt;
     int64_t cnt_words;
 };
+// Outlier detection and row quantization in one cooperative launch: column
+// flags of every row, a grid barrier, then codes/scales/outlier gathers.
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 
 struct GemmArgs {
@@ -270,6 +271,20 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// 2-D tiled TMA store shared -> global (bulk-group completion). Elements of
+// the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most one committed store group may still be reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// Every committed store group has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // --- CTA pairs (cluster of 2) and the 2-SM tensor-core instructions -------
 

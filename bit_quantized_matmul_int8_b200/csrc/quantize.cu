@@ -7,9 +7,11 @@
 //
 // Kernels (all HBM-bound streaming passes with 16-byte coalesced loads):
 //   prepare_weight_kernel  W [N,K] -> CB, SCB          (one warp per row)
-//   outlier_flags_kernel   X [M,K] -> partial column bitmaps (phase A)
-//   quantize_kernel        X, bitmaps -> O, CA, SCA, Xo; gathers Wo; clears
-//                          the split-K buffers of the GEMV      (phase B)
+//   quantize_kernel        one cooperative launch: phase A ORs the outlier
+//                          columns of every row into a bitmap, a grid
+//                          barrier, then phase B writes O, CA, SCA, Xo,
+//                          gathers Wo and clears the split-K buffers of the
+//                          GEMV
 //
 // Exactness: |x| >= threshold is decided on the fp16 bit pattern against the
 // smallest fp16 pattern whose value reaches the fp32 threshold (the map from
@@ -18,6 +20,7 @@
 // rint(x * fp32(127 / absmax)) with __fdiv_rn / __fmul_rn / __float2int_rn:
 // one IEEE rounding per step, ties to even, never contracted into an FMA.
 #include <algorithm>
+#include <mutex>
 
 #include "int8lt_internal.cuh"
 
@@ -28,10 +31,18 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
-// rint(x * s) with s = fp32(127 / absmax) and |x| <= absmax. No clamp is
-// needed: |x * s| <= 127 * (1 + 2^-23) before rounding, so the fp32 product
-// rounds to at most 127.00001 and rint gives at most 127 in magnitude.
-__device__ __forceinline__ int32_t quant_code(float x, float s) { return __float2int_rn(__fmul_rn(x, s)); }
+// Code of x: rint(fp32(x * s)) with s = fp32(127 / absmax) and |x| <= absmax.
+// No clamp is needed: |x * s| <= 127 * (1 + 2^-23) before rounding, so the
+// fp32 product is at most 127.00001 and its rint at most 127 in magnitude.
+// rint(v) for |v| < 2^22 is taken by adding 1.5 * 2^23 in fp32: the sum lies
+// in [2^23, 2^24), where consecutive fp32 values are consecutive integers, so
+// IEEE round-to-nearest-even of the addition is rint(v) + 1.5 * 2^23; the low
+// byte of the sum's bit pattern is then the low byte of rint(v) (two's
+// complement), because 1.5 * 2^23 = 0xC00000 has a zero low byte. Both steps
+// are separate _rn operations, so they are never fused into one FMA.
+__device__ __forceinline__ uint32_t code_bits(float x, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(x, s), 12582912.0f));
+}
 
 __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
 #pragma unroll
@@ -46,10 +57,9 @@ __device__ __forceinline__ uint32_t vec_absmax_bits(uint4 v) {
     return max(m & 0xffffu, m >> 16);
 }
 
-__device__ __forceinline__ uint32_t pack4(int32_t a, int32_t b, int32_t c, int32_t d) {
-    // low bytes of four small integers -> one word (byte 0 = a)
-    return __byte_perm(__byte_perm((uint32_t)a, (uint32_t)b, 0x0040), __byte_perm((uint32_t)c, (uint32_t)d, 0x0040),
-                       0x5410);
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    // low bytes of four words -> one word (byte 0 = a)
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 __device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
@@ -57,8 +67,8 @@ __device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
     float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
     float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
     uint2 r;
-    r.x = pack4(quant_code(f0.x, s), quant_code(f0.y, s), quant_code(f1.x, s), quant_code(f1.y, s));
-    r.y = pack4(quant_code(f2.x, s), quant_code(f2.y, s), quant_code(f3.x, s), quant_code(f3.y, s));
+    r.x = pack4(code_bits(f0.x, s), code_bits(f0.y, s), code_bits(f1.x, s), code_bits(f1.y, s));
+    r.y = pack4(code_bits(f2.x, s), code_bits(f2.y, s), code_bits(f3.x, s), code_bits(f3.y, s));
     return r;
 }
 
@@ -90,64 +100,9 @@ prepare_weight_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int8_t
             uint2 *c2 = reinterpret_cast<uint2 *>(cb);
             for (int64_t v = lane; v < K / 8; v += 32) c2[v] = quant_vec8(__ldg(w4 + v), s);
         } else {
-            for (int64_t k = lane; k < K; k += 32) cb[k] = (int8_t)quant_code(__half2float(w[k]), s);
+            for (int64_t k = lane; k < K; k += 32) cb[k] = (int8_t)(code_bits(__half2float(w[k]), s) & 0xffu);
         }
         if (lane == 0) SCB[j] = a;
-    }
-}
-
-// ------------------------------------------------------- phase A: flags ----
-
-// Block (x, y): columns [64x, 64x + 64), row chunk y. Lane l reads the 16-byte
-// vector (l & 7) of row (4 * warp + (l >> 3)) + 32 i of the chunk, 8 rows
-// in flight per thread. Writes flags[y][2x], flags[y][2x + 1] (no atomics).
-constexpr int kFlagUnroll = 8;
-
-__global__ void __launch_bounds__(kThreads)
-outlier_flags_kernel(const __half *__restrict__ X, int64_t M, int64_t K, uint32_t tbits,
-                     uint32_t *__restrict__ flags, int64_t kwords) {
-    __shared__ uint32_t sflags[2];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (threadIdx.x < 2) sflags[threadIdx.x] = 0;
-    __syncthreads();
-    const int64_t c0 = (int64_t)blockIdx.x * kColsPerFlagCta + (lane & 7) * 8;
-    const int64_t rows_per = ceil_div(M, gridDim.y);
-    const int64_t r1 = min(M, (int64_t)blockIdx.y * rows_per + rows_per);
-    const uint32_t t2 = tbits | (tbits << 16);
-    // hit[w]: per 16-bit half 0xffff where some |x| >= threshold; half 0 of
-    // word w is column 2w of the lane's 8 columns, half 1 is column 2w + 1.
-    uint32_t hit[4] = {0u, 0u, 0u, 0u};
-    if (c0 < K) {
-        const __half *xc = X + c0;
-        for (int64_t r = (int64_t)blockIdx.y * rows_per + warp * 4 + (lane >> 3); r < r1;
-             r += kFlagUnroll * 32) {
-            uint4 v[kFlagUnroll];
-#pragma unroll
-            for (int u = 0; u < kFlagUnroll; ++u) {
-                const int64_t ru = r + u * 32;
-                v[u] = ru < r1 ? __ldg(reinterpret_cast<const uint4 *>(xc + ru * K)) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < kFlagUnroll; ++u) {
-                hit[0] |= __vcmpgeu2(v[u].x & 0x7fff7fffu, t2);
-                hit[1] |= __vcmpgeu2(v[u].y & 0x7fff7fffu, t2);
-                hit[2] |= __vcmpgeu2(v[u].z & 0x7fff7fffu, t2);
-                hit[3] |= __vcmpgeu2(v[u].w & 0x7fff7fffu, t2);
-            }
-        }
-    }
-    // Zero-padded rows compare as |0| >= T, true only for T = 0, where every
-    // column is an outlier anyway (and then only real columns are kept).
-    uint32_t byte = 0;  // bit j: column c0 + j is an outlier column
-#pragma unroll
-    for (int w = 0; w < 4; ++w) byte |= ((hit[w] & 1u) << (2 * w)) | (((hit[w] >> 16) & 1u) << (2 * w + 1));
-    byte |= __shfl_xor_sync(0xffffffffu, byte, 8);
-    byte |= __shfl_xor_sync(0xffffffffu, byte, 16);
-    if (lane < 8 && byte) atomicOr(&sflags[lane >> 2], byte << ((lane & 3) * 8));
-    __syncthreads();
-    if (threadIdx.x < 2) {
-        const int64_t word = (int64_t)blockIdx.x * 2 + threadIdx.x;
-        if (word < kwords) flags[(int64_t)blockIdx.y * kwords + word] = sflags[threadIdx.x];
     }
 }
 
@@ -317,25 +272,120 @@ __device__ void quantize_rows_team(const QuantizeArgs &a, const uint32_t *bits, 
     }
 }
 
+// Outlier byte of a 16-byte vector: bit j set where |x_j| >= threshold,
+// decided on the fp16 magnitude bits against the threshold pattern.
+__device__ __forceinline__ uint32_t outlier_byte(uint4 v, uint32_t t2) {
+    const uint32_t h0 = __vcmpgeu2(v.x & 0x7fff7fffu, t2), h1 = __vcmpgeu2(v.y & 0x7fff7fffu, t2);
+    const uint32_t h2 = __vcmpgeu2(v.z & 0x7fff7fffu, t2), h3 = __vcmpgeu2(v.w & 0x7fff7fffu, t2);
+    return (h0 & 1u) | ((h0 >> 15) & 2u) | ((h1 & 1u) << 2) | ((h1 >> 13) & 8u) | ((h2 & 1u) << 4) |
+           ((h2 >> 11) & 32u) | ((h3 & 1u) << 6) | ((h3 >> 9) & 128u);
+}
+
+// Phase A for one team's rows: OR the rows' outlier bits into the CTA bitmap.
+template <int T, int V>
+__device__ void flag_rows_team(const QuantizeArgs &a, uint32_t *bits, int teams_total) {
+    const int teams = kThreads / T;
+    const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
+    const int64_t nvec = a.K / 8;
+    const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
+    for (int64_t r = (int64_t)blockIdx.x * teams + team; r < a.M; r += teams_total) {
+        const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
+        if constexpr (V > 0) {
+            uint4 x[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int64_t v = tl + (int64_t)i * T;
+                x[i] = v < nvec ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int64_t v = tl + (int64_t)i * T;
+                const uint32_t b = v < nvec ? outlier_byte(x[i], t2) : 0u;
+                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
+            }
+        } else {
+            for (int64_t v = tl; v < nvec; v += T) {
+                const uint32_t b = outlier_byte(__ldg(x4 + v), t2);
+                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier of the cooperative launch. The last CTA to arrive resets
+// the count and advances the generation, which releases the others; every
+// wait is bounded. Returns false (and records a timeout) if it ran out.
+__device__ bool grid_barrier(WsHeader *h, uint32_t gen) {
+    __shared__ uint32_t s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t ok = 1;
+        __threadfence();
+        const uint32_t old = atomicAdd(&h->bar_count, 1u);
+        if (old == gridDim.x - 1) {
+            atomicExch(&h->bar_count, 0u);
+            __threadfence();
+            atomicExch(&h->qgen, gen + 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_u32(&h->qgen) == gen) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    ok = 0;
+                    record_timeout(&h->status);
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
 template <int T, int V>
 __global__ void __launch_bounds__(kThreads, 2)
-quantize_kernel(QuantizeArgs a, int64_t kwords, int row_ctas) {
+quantize_kernel(QuantizeArgs a, int64_t kwords) {
     extern __shared__ uint32_t smem[];
     __shared__ uint32_t red[kWarps];
+    __shared__ uint32_t s_gen;
     uint32_t *bits = smem;                                         // [kwords]
     int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
-    // O = OR of the phase-A partial bitmaps.
+    const int teams_total = gridDim.x * (kThreads / T);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    // This launch's bitmap is bitmaps[gen & 1]; the previous launch zeroed it.
+    if (threadIdx.x == 0) s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
+    for (int64_t w = threadIdx.x; w < kwords; w += kThreads) bits[w] = 0;
+    __syncthreads();
+    const uint32_t gen = s_gen;
+    uint32_t *cur = a.bitmaps + (gen & 1u) * kMaxKwords;
+    uint32_t *nxt = a.bitmaps + ((gen + 1u) & 1u) * kMaxKwords;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
+        nxt[i] = 0;
+
+    // Phase A: O = { h : some |X[i,h]| >= threshold } over every row.
+    flag_rows_team<T, V>(a, bits, teams_total);
+    __syncthreads();
+    for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
+        if (bits[w]) atomicOr(&cur[w], bits[w]);
+    if (!grid_barrier(a.hdr, gen)) return;  // every CTA waits in the same barrier
+
+    // Phase B: codes, scales, outlier activations; outlier-weight gather.
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
-        uint32_t v = 0;
-        for (int64_t c = 0; c < a.flag_chunks; ++c) v |= a.flags[c * kwords + w];
+        uint32_t v = __ldcg(&cur[w]);
         if (w == kwords - 1 && (a.K & 31)) v &= (1u << (a.K & 31)) - 1u;
         bits[w] = v;
     }
     __syncthreads();
     const int32_t n_out = build_prefix(bits, prefix, kwords);
     const int32_t n16 = (n_out + 15) & ~15;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-
     if (blockIdx.x == 0) {
         if (threadIdx.x == 0 && a.n_outliers) *a.n_outliers = n_out;
         if (a.outlier_idx) {
@@ -349,36 +399,30 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int row_ctas) {
             }
         }
     }
-
-    if ((int)blockIdx.x < row_ctas) {
-        quantize_rows_team<T, V>(a, bits, prefix, n_out, row_ctas, red);
-    } else {
-        // Extra blocks: outlier-weight gather and split-K buffer clearing.
-        const int64_t eb = blockIdx.x - row_ctas, neb = gridDim.x - row_ctas;
-        if (a.Wo) {
-            for (int64_t j = eb * kWarps + warp; j < a.N; j += neb * kWarps) {
-                __half *wo = a.Wo + j * a.kcap;
-                for (int32_t t = lane; t < n16; t += 32) {
-                    __half val = __float2half_rn(0.f);
-                    if (t < n_out) {
-                        int64_t col = outlier_column(bits, prefix, kwords, t);
-                        if (a.W_outlier) {
-                            val = a.W_outlier[j * a.K + col];
-                        } else {
-                            float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
-                            val = __float2half_rn(__fdiv_rn(p, 127.f));
-                        }
+    quantize_rows_team<T, V>(a, bits, prefix, n_out, gridDim.x, red);
+    if (a.Wo) {
+        for (int64_t j = (int64_t)blockIdx.x * kWarps + warp; j < a.N; j += (int64_t)gridDim.x * kWarps) {
+            __half *wo = a.Wo + j * a.kcap;
+            for (int32_t t = lane; t < n16; t += 32) {
+                __half val = __float2half_rn(0.f);
+                if (t < n_out) {
+                    const int64_t col = outlier_column(bits, prefix, kwords, t);
+                    if (a.W_outlier) {
+                        val = a.W_outlier[j * a.K + col];
+                    } else {
+                        const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
+                        val = __float2half_rn(__fdiv_rn(p, 127.f));
                     }
-                    wo[t] = val;
                 }
+                wo[t] = val;
             }
         }
-        const int64_t tid = eb * kThreads + threadIdx.x, nth = neb * kThreads;
-        if (a.acc)
-            for (int64_t i = tid; i < a.acc_words; i += nth) a.acc[i] = 0;
-        if (a.cnt)
-            for (int64_t i = tid; i < a.cnt_words; i += nth) a.cnt[i] = 0;
     }
+    const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x, nth = (int64_t)gridDim.x * kThreads;
+    if (a.acc)
+        for (int64_t i = tid; i < a.acc_words; i += nth) a.acc[i] = 0;
+    if (a.cnt)
+        for (int64_t i = tid; i < a.cnt_words; i += nth) a.cnt[i] = 0;
 }
 
 }  // namespace
@@ -406,26 +450,57 @@ cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t 
     return cudaGetLastError();
 }
 
-cudaError_t launch_outlier_flags(const __half *X, int64_t M, int64_t K, uint16_t tbits,
-                                 uint32_t *flags, int64_t flag_chunks, cudaStream_t s) {
-    dim3 grid((unsigned)ceil_div(K, kColsPerFlagCta), (unsigned)flag_chunks);
-    outlier_flags_kernel<<<grid, kThreads, 0, s>>>(X, M, K, tbits, flags, ceil_div(K, 32));
-    return cudaGetLastError();
-}
-
 namespace {
 
+// Resident CTAs of one kernel instance on the current device (for the
+// cooperative grid size), computed once per device.
 template <int T, int V>
-cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, int row_ctas, int extra,
-                               cudaStream_t s) {
+cudaError_t resident_ctas(size_t smem, int *out) {
+    static std::once_flag once[64];
+    static int count[64];
+    static cudaError_t err[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    dev &= 63;
+    std::call_once(once[dev], [&] {
+        int per_sm = 0, sms = 0;
+        err[dev] = cudaFuncSetAttribute(quantize_kernel<T, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)(2 * kMaxKwords * 4));
+        if (err[dev] == cudaSuccess)
+            err[dev] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel<T, V>, kThreads,
+                                                                     2 * kMaxKwords * 4);
+        if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        count[dev] = per_sm * sms;
+    });
+    (void)smem;
+    *out = count[dev];
+    return err[dev];
+}
+
+template <int T, int V>
+cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, cudaStream_t s) {
     const size_t smem = (size_t)kwords * 8;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(quantize_kernel<T, V>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    quantize_kernel<T, V><<<row_ctas + extra, kThreads, smem, s>>>(a, kwords, row_ctas);
-    return cudaGetLastError();
+    int max_ctas = 0;
+    if (cudaError_t e = resident_ctas<T, V>(smem, &max_ctas)) return e;
+    if (max_ctas <= 0) return cudaErrorInvalidConfiguration;
+    const int teams = kThreads / T;
+    // Enough teams for every row where possible; the grid barrier needs every
+    // CTA resident at once, which the cooperative launch guarantees.
+    int64_t want = ceil_div(a.M, teams);
+    if (a.Wo) want = std::max<int64_t>(want, std::min<int64_t>(ceil_div(a.N, kWarps), 148));
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_kernel<T, V>, a, kwords);
 }
 
 }  // namespace
@@ -433,20 +508,20 @@ cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, int row_ct
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     const int64_t kwords = ceil_div(a.K, 32);
     const int64_t nvec = a.K / 8;
-    // Row team: one warp per row up to K = 4096 (16 vectors per lane), four
-    // warps per row up to K = 16384; longer rows are read twice.
-    const int T = nvec <= 128 ? 32 : 128;
-    const int teams = kThreads / T;
-    int row_ctas = (int)std::min<int64_t>(ceil_div(a.M, teams), 148 * 8);
-    int extra = 0;
-    if (a.Wo) extra = (int)std::min<int64_t>(ceil_div(a.N, 64), 128);
-    else if (a.acc) extra = (int)std::min<int64_t>(ceil_div(a.acc_words, 4096) + 1, 148);
+    // Row team: one warp per row up to K = 4096 (up to 16 loads in flight per
+    // lane, and every row of a 2048-token batch in flight at once), four warps
+    // per row up to K = 16384 (the row stays in registers); longer rows are
+    // read twice.
+    const int T = nvec <= 32 * 16 ? 32 : 128;
     const int64_t v = ceil_div(nvec, T);
-    if (T == 32) return launch_quantize_tv<32, 4>(a, kwords, row_ctas, extra, s);
-    if (v <= 4) return launch_quantize_tv<128, 4>(a, kwords, row_ctas, extra, s);
-    if (v <= 8) return launch_quantize_tv<128, 8>(a, kwords, row_ctas, extra, s);
-    if (v <= 16) return launch_quantize_tv<128, 16>(a, kwords, row_ctas, extra, s);
-    return launch_quantize_tv<128, 0>(a, kwords, row_ctas, extra, s);
+    if (T == 32) {
+        if (v <= 4) return launch_quantize_tv<32, 4>(a, kwords, s);
+        if (v <= 8) return launch_quantize_tv<32, 8>(a, kwords, s);
+        return launch_quantize_tv<32, 16>(a, kwords, s);
+    }
+    if (v <= 8) return launch_quantize_tv<128, 8>(a, kwords, s);
+    if (v <= 16) return launch_quantize_tv<128, 16>(a, kwords, s);
+    return launch_quantize_tv<128, 0>(a, kwords, s);
 }
 
 }  // namespace int8lt

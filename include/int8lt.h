@@ -83,8 +83,11 @@ int int8lt_version(void);
 size_t int8lt_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * Clear the workspace's device status word (stream-ordered). Call once after
- * allocating a workspace; int8lt_read_device_status also clears it.
+ * Prepare a freshly allocated workspace (stream-ordered): clears its first
+ * 34 KB (device status word, outlier count, the quantize pass's launch
+ * counter and its column bitmaps). Call once after allocating a workspace,
+ * before its first use; later calls keep it consistent by themselves.
+ * int8lt_read_device_status clears the status word alone.
  */
 int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
