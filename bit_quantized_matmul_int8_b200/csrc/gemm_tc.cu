@@ -49,7 +49,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kEpiOutlierMax = 32;
+constexpr int kEpiOutlierMax = 24;  // largest |O| whose product runs on the CUDA cores
 constexpr int kEpiBarrier = 1;            // named barrier of the epilogue warps
 constexpr uint16_t kPairMask = 0x3;       // both CTAs of the cluster
 
@@ -80,14 +80,116 @@ constexpr size_t kOffStage = kSmemTiles;                         // [kEpiWarps][
 constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * 2 * kStoreBufBytes;
 constexpr size_t kOffScb = kOffCtrl + 256;
 constexpr size_t kOffBias = kOffScb + BN * 4;
-constexpr size_t kOffWo = kOffBias + BN * 4;                     // fp16 [kEpiOutlierMax][BN]
-constexpr size_t kSmemUsed = kOffWo + (size_t)kEpiOutlierMax * BN * 2;
+constexpr size_t kOffWo = kOffBias + BN * 4;                     // fp32 [kEpiOutlierMax][BN]
+constexpr size_t kSmemUsed = kOffWo + (size_t)kEpiOutlierMax * BN * 4;
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kSmemUsed;
 static_assert(sizeof(Ctrl) <= 256, "control block");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync %0, %1;" ::"r"(kEpiBarrier), "r"(kEpiThreads) : "memory");
+}
+
+// Epilogue of one tile for one warp: 32 rows (TMEM lanes) x 128 columns, in
+// chunks of 32. kMmaOut: the outlier product P is in TMEM (fp32, 256 columns
+// after the int32 sums); otherwise it is computed here from Xo and Wo.
+template <bool kMmaOut>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem, uint32_t lane_base, int buf, int hcol,
+                                              int q, int lane, int ew, uint32_t rank, bool row_ok, int64_t row,
+                                              float rs, int64_t n0, int64_t m0, int n_out, const float *s_scb,
+                                              const float *s_bias, const float *s_wo, uint8_t *s_stage, int &sbuf,
+                                              Ctrl *ctrl, const CUtensorMap *tmY,
+                                              const uint4 (&xo_v)[kEpiOutlierMax / 8]) {
+    const bool cuda_out = !kMmaOut && n_out > 0;
+    // This row's outlier activations (CUDA-core outlier product), fp16.
+    const __half *xo = reinterpret_cast<const __half *>(xo_v);
+    const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
+    for (int cc = 0; cc < 128; cc += 32) {
+        const int c = hcol * 128 + cc;  // column within the tile
+        uint32_t acc[32], po[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+        if constexpr (kMmaOut) tmem_ld_32x32b_x32(tmem + lane_base + 256 + col0 + cc, po);
+        tmem_ld_wait();
+        if (cc == 96) {
+            // Every TMEM read of this buffer is done: hand it back to
+            // the leader's MMA warp.
+            tc_fence_before();
+            if (lane == 0) {
+                const uint32_t eb = smem_u32(&ctrl->acc_empty[buf]);
+                if (rank == 0) mbar_arrive(eb); else mbar_arrive_cluster(mapa_shared(eb, 0));
+            }
+        }
+        if (n0 + c >= a.N) continue;  // whole chunk past the last column
+        if (a.C32) {
+            if (!row_ok) continue;
+            int32_t *dst = a.C32 + row * a.N + n0 + c;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                if (n0 + c + 4 * v < a.N)
+                    reinterpret_cast<int4 *>(dst)[v] =
+                        make_int4((int)acc[4 * v], (int)acc[4 * v + 1], (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
+            continue;
+        }
+        // y = C * SCA / 127^2 * SCB + bias (+ P), two columns per
+        // packed fp32x2 operation (each lane rounds like fmaf/fmul).
+        float2 y2[16];
+        const float2 rs2 = make_float2(rs, rs);
+        const float4 *sc4 = reinterpret_cast<const float4 *>(s_scb + c);
+        const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias + c);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const float4 sc = sc4[v], bi = bi4[v];
+            const float2 c01 = __fmul2_rn(make_float2((float)(int32_t)acc[4 * v], (float)(int32_t)acc[4 * v + 1]), rs2);
+            const float2 c23 =
+                __fmul2_rn(make_float2((float)(int32_t)acc[4 * v + 2], (float)(int32_t)acc[4 * v + 3]), rs2);
+            y2[2 * v] = __ffma2_rn(c01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
+            y2[2 * v + 1] = __ffma2_rn(c23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
+        }
+        if constexpr (kMmaOut) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                y2[k] = __fadd2_rn(y2[k], make_float2(__uint_as_float(po[2 * k]), __uint_as_float(po[2 * k + 1])));
+        }
+        if (!kMmaOut && cuda_out) {
+#pragma unroll
+            for (int t = 0; t < (kMmaOut ? 1 : kEpiOutlierMax); ++t) {
+                if (t >= n_out) break;  // uniform across the CTA
+                const float xt = __half2float(xo[t]);
+                const float2 xv = make_float2(xt, xt);
+                const float4 *w4 = reinterpret_cast<const float4 *>(s_wo + t * BN + c);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 wv = w4[v];
+                    y2[2 * v] = __ffma2_rn(xv, make_float2(wv.x, wv.y), y2[2 * v]);
+                    y2[2 * v + 1] = __ffma2_rn(xv, make_float2(wv.z, wv.w), y2[2 * v + 1]);
+                }
+            }
+        }
+        uint32_t packed[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            __half2 h = __float22half2_rn(y2[k]);
+            packed[k] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        // Stage the warp's 32 x 32 box in shared memory (64-byte swizzle:
+        // 16-byte chunk i of row r sits at chunk i ^ ((r >> 1) & 3), which
+        // keeps the four stores of each row conflict-free) and hand it to
+        // the TMA engine. Rows and columns past M and N are clipped by it.
+        if (lane == 0) bulk_wait_read_1();  // this buffer's previous store has read it
+        __syncwarp();
+        uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
+                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, smem_u32(box), (int32_t)(n0 + c), (int32_t)(m0 + q * 32));
+            bulk_commit_group();
+        }
+        sbuf ^= 1;
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -102,7 +204,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem + kOffCtrl);
     float *s_scb = reinterpret_cast<float *>(smem + kOffScb);
     float *s_bias = reinterpret_cast<float *>(smem + kOffBias);
-    __half *s_wo = reinterpret_cast<__half *>(smem + kOffWo);
+    float *s_wo = reinterpret_cast<float *>(smem + kOffWo);
     uint8_t *s_stage = smem + kOffStage;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,6 +358,25 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int64_t n0 = (int64_t)(tile / num_m_tiles) * BN;
             const int buf = it % nbuf;
             const uint32_t use = (uint32_t)(it / nbuf);
+            // Fetch this tile's column data (thread et owns column n0 + et)
+            // and this thread's row data into registers while the MMAs are
+            // still running: 16-byte loads, all issued before any wait.
+            const int64_t col = n0 + et;
+            const bool col_ok = !a.C32 && col < a.N;
+            const float scb_v = col_ok ? a.SCB[col] : 0.f;
+            const float bias_v = (col_ok && a.bias) ? __half2float(a.bias[col]) : 0.f;
+            const int64_t row = m0 + q * 32 + lane;
+            const bool row_ok = row < a.M;
+            const float sca_v = (row_ok && a.SCA) ? a.SCA[row] : 0.f;
+            uint4 wo_v[kEpiOutlierMax / 8], xo_v[kEpiOutlierMax / 8];
+#pragma unroll
+            for (int v = 0; v < kEpiOutlierMax / 8; ++v) {
+                const bool need = cuda_out && 8 * v < n_out;
+                wo_v[v] = (need && col_ok) ? *reinterpret_cast<const uint4 *>(a.Wo + col * a.kcap + 8 * v)
+                                           : make_uint4(0, 0, 0, 0);
+                xo_v[v] = (need && row_ok) ? *reinterpret_cast<const uint4 *>(a.Xo + row * a.kcap + 8 * v)
+                                           : make_uint4(0, 0, 0, 0);
+            }
             // Wait for the accumulator, then decide together whether to go
             // on: every epilogue warp votes before the barrier and reads the
             // same slot after it, so all of them leave the loop together.
@@ -271,124 +392,24 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 break;
             }
             if (!a.C32) {
-                for (int c = et; c < BN; c += kEpiThreads) {
-                    const int64_t j = n0 + c;
-                    s_scb[c] = j < a.N ? a.SCB[j] : 0.f;
-                    s_bias[c] = (a.bias && j < a.N) ? __half2float(a.bias[j]) : 0.f;
-                }
+                s_scb[et] = scb_v;
+                s_bias[et] = bias_v;
                 if (cuda_out) {
-                    const int n16 = (n_out + 15) & ~15;
-                    for (int i = et; i < n16 * BN; i += kEpiThreads) {
-                        const int t = i / BN, c = i % BN;
-                        const int64_t j = n0 + c;
-                        s_wo[t * BN + c] = j < a.N ? a.Wo[j * a.kcap + t] : __float2half_rn(0.f);
-                    }
+                    const __half *wh = reinterpret_cast<const __half *>(wo_v);
+#pragma unroll
+                    for (int t = 0; t < kEpiOutlierMax; ++t)
+                        if (t < n_out) s_wo[t * BN + et] = __half2float(wh[t]);
                 }
             }
             epi_sync();
             tc_fence_after();
-            const int64_t row = m0 + q * 32 + lane;
-            const bool row_ok = row < a.M;
-            const float rs = (row_ok && a.SCA) ? a.SCA[row] * (1.0f / 16129.0f) : 0.f;
-            // This row's outlier activations (CUDA-core outlier product).
-            __half2 xo2[kEpiOutlierMax / 2];
-            if (cuda_out) {
-#pragma unroll
-                for (int t = 0; t < kEpiOutlierMax / 2; ++t)
-                    xo2[t] = (row_ok && 2 * t < n_out)
-                                 ? *reinterpret_cast<const __half2 *>(a.Xo + row * a.kcap + 2 * t)
-                                 : __floats2half2_rn(0.f, 0.f);
-            }
-            const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
-            for (int cc = 0; cc < 128; cc += 32) {
-                const int c = hcol * 128 + cc;  // column within the tile
-                uint32_t acc[32], po[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
-                if (mma_out) tmem_ld_32x32b_x32(tmem + lane_base + 256 + col0 + cc, po);
-                tmem_ld_wait();
-                if (cc == 96) {
-                    // Every TMEM read of this buffer is done: hand it back to
-                    // the leader's MMA warp.
-                    tc_fence_before();
-                    if (lane == 0) {
-                        const uint32_t eb = smem_u32(&ctrl->acc_empty[buf]);
-                        if (rank == 0) mbar_arrive(eb); else mbar_arrive_cluster(mapa_shared(eb, 0));
-                    }
-                }
-                if (n0 + c >= a.N) continue;  // whole chunk past the last column
-                if (a.C32) {
-                    if (!row_ok) continue;
-                    int32_t *dst = a.C32 + row * a.N + n0 + c;
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        if (n0 + c + 4 * v < a.N)
-                            reinterpret_cast<int4 *>(dst)[v] =
-                                make_int4((int)acc[4 * v], (int)acc[4 * v + 1], (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
-                    continue;
-                }
-                float y[32];
-                const float4 *sc4 = reinterpret_cast<const float4 *>(s_scb + c);
-                const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias + c);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 sc = sc4[v], bi = bi4[v];
-                    y[4 * v + 0] = fmaf((float)(int32_t)acc[4 * v + 0] * rs, sc.x, bi.x);
-                    y[4 * v + 1] = fmaf((float)(int32_t)acc[4 * v + 1] * rs, sc.y, bi.y);
-                    y[4 * v + 2] = fmaf((float)(int32_t)acc[4 * v + 2] * rs, sc.z, bi.z);
-                    y[4 * v + 3] = fmaf((float)(int32_t)acc[4 * v + 3] * rs, sc.w, bi.w);
-                }
-                if (mma_out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(po[j]);
-                }
-                if (cuda_out) {
-#pragma unroll
-                    for (int t2 = 0; t2 < kEpiOutlierMax / 2; ++t2) {
-                        if (2 * t2 >= n_out) break;  // uniform across the CTA
-                        const float2 xf = __half22float2(xo2[t2]);
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const float xv = h ? xf.y : xf.x;
-                            const uint4 *w4 = reinterpret_cast<const uint4 *>(s_wo + (2 * t2 + h) * BN + c);
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                const uint4 wv = w4[v];
-                                const __half2 *wh = reinterpret_cast<const __half2 *>(&wv);
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    const float2 wf = __half22float2(wh[u]);
-                                    y[8 * v + 2 * u] = fmaf(xv, wf.x, y[8 * v + 2 * u]);
-                                    y[8 * v + 2 * u + 1] = fmaf(xv, wf.y, y[8 * v + 2 * u + 1]);
-                                }
-                            }
-                        }
-                    }
-                }
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    __half2 h = __floats2half2_rn(y[j], y[j + 1]);
-                    packed[j >> 1] = *reinterpret_cast<uint32_t *>(&h);
-                }
-                // Stage the warp's 32 x 32 box in shared memory (64-byte swizzle:
-                // 16-byte chunk i of row r sits at chunk i ^ ((r >> 1) & 3), which
-                // keeps the four stores of each row conflict-free) and hand it to
-                // the TMA engine. Rows and columns past M and N are clipped by it.
-                if (lane == 0) bulk_wait_read_1();  // this buffer's previous store has read it
-                __syncwarp();
-                uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
-                        make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, smem_u32(box), (int32_t)(n0 + c), (int32_t)(m0 + q * 32));
-                    bulk_commit_group();
-                }
-                sbuf ^= 1;
-            }
+            const float rs = sca_v * (1.0f / 16129.0f);
+            if (mma_out)
+                epilogue_tile<true>(a, tmem, lane_base, buf, hcol, q, lane, ew, rank, row_ok, row, rs, n0, m0, n_out,
+                                    s_scb, s_bias, s_wo, s_stage, sbuf, ctrl, &tmY, xo_v);
+            else
+                epilogue_tile<false>(a, tmem, lane_base, buf, hcol, q, lane, ew, rank, row_ok, row, rs, n0, m0, n_out,
+                                     s_scb, s_bias, s_wo, s_stage, sbuf, ctrl, &tmY, xo_v);
         }
         if (lane == 0) bulk_wait_all();  // every store of this warp has finished
     }

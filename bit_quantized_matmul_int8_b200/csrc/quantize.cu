@@ -225,6 +225,36 @@ __device__ __forceinline__ uint32_t team_max(uint32_t v, uint32_t *red, int team
 
 // One row per team of T threads; the team's row is held in V 16-byte
 // registers per thread (V * T * 8 >= K), or re-read when V == 0.
+// Phase B of one row held in registers (V > 0): masked absmax over the team,
+// codes, scale and outlier activations. Every thread of the team calls it.
+template <int T, int V>
+__device__ __forceinline__ void quantize_row_regs(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
+                                                  int32_t n_out, const uint4 (&x)[V], int64_t r, bool valid,
+                                                  uint32_t *red, int team, int tl) {
+    const int64_t nvec = a.K / 8;
+    const int32_t n16 = (n_out + 15) & ~15;
+    uint32_t amax = 0;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int64_t v = tl + (int64_t)i * T;
+        if (valid && v < nvec) amax = max(amax, masked_absmax_bits(x[i], vec_mask(bits, v)));
+    }
+    amax = team_max<T>(amax, red, team);
+    if (!valid) return;
+    const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+    const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+    uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+    __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int64_t v = tl + (int64_t)i * T;
+        if (v < nvec) ca2[v] = quant_masked(x[i], vec_mask(bits, v), s, v, bits, prefix, xo);
+    }
+    if (xo)
+        for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
+    if (tl == 0) a.SCA[r] = sa;
+}
+
 template <int T, int V>
 __device__ void quantize_rows_team(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
                                    int32_t n_out, int row_ctas, uint32_t *red) {
@@ -329,9 +359,10 @@ __device__ bool grid_barrier(WsHeader *h, uint32_t gen) {
         __threadfence();
         const uint32_t old = atomicAdd(&h->bar_count, 1u);
         if (old == gridDim.x - 1) {
-            atomicExch(&h->bar_count, 0u);
-            __threadfence();
+            // Release the waiters first; the count is reset for the next
+            // launch, which stream order keeps behind this one.
             atomicExch(&h->qgen, gen + 1u);
+            atomicExch(&h->bar_count, 0u);
         } else {
             const uint64_t t0 = globaltimer_ns();
             while (ld_acquire_u32(&h->qgen) == gen) {
@@ -370,8 +401,35 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
         nxt[i] = 0;
 
+    // With one row (or none) per team, the team keeps its row in registers
+    // from phase A to phase B instead of reading it twice.
+    constexpr int kTeams = kThreads / T;
+    const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
+    const bool one_round = V > 0 && a.M <= teams_total;
+    const int64_t my_row = (int64_t)blockIdx.x * kTeams + team;
+    uint4 xr[V > 0 ? V : 1];
+
     // Phase A: O = { h : some |X[i,h]| >= threshold } over every row.
-    flag_rows_team<T, V>(a, bits, teams_total);
+    if (one_round) {
+        if constexpr (V > 0) {
+            const int64_t nvec = a.K / 8;
+            const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
+            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + my_row * a.K);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int64_t v = tl + (int64_t)i * T;
+                xr[i] = (my_row < a.M && v < nvec) ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int64_t v = tl + (int64_t)i * T;
+                const uint32_t b = (my_row < a.M && v < nvec) ? outlier_byte(xr[i], t2) : 0u;
+                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
+            }
+        }
+    } else {
+        flag_rows_team<T, V>(a, bits, teams_total);
+    }
     __syncthreads();
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
         if (bits[w]) atomicOr(&cur[w], bits[w]);
@@ -399,7 +457,11 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
             }
         }
     }
-    quantize_rows_team<T, V>(a, bits, prefix, n_out, gridDim.x, red);
+    if (one_round) {
+        if constexpr (V > 0) quantize_row_regs<T, V>(a, bits, prefix, n_out, xr, my_row, my_row < a.M, red, team, tl);
+    } else {
+        quantize_rows_team<T, V>(a, bits, prefix, n_out, gridDim.x, red);
+    }
     if (a.Wo) {
         for (int64_t j = (int64_t)blockIdx.x * kWarps + warp; j < a.N; j += (int64_t)gridDim.x * kWarps) {
             __half *wo = a.Wo + j * a.kcap;
