@@ -27,7 +27,7 @@ EXPORTS = [
     "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
-    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_wait_timeout",
+    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout",
 ]
 
 
@@ -56,6 +56,7 @@ _SIGS = {
     "int8lt_forward_static_scratch": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P]),
     "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
+    "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
 }
 
 

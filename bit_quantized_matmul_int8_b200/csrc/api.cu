@@ -25,9 +25,11 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
     L.xo = off;    off += align_up((size_t)M * L.kcap * 2);
     if (M > kDecodeMaxM) {
         L.wo = off; off += align_up((size_t)N * L.kcap * 2);
+        L.sk = off; off += align_up((size_t)kSkMaxPairs * 2 * kSkPartialBytes);
         L.acc = L.cnt = SIZE_MAX;
     } else {
         L.wo = SIZE_MAX;
+        L.sk = SIZE_MAX;
         L.acc = off; off += align_up((size_t)N * 16 * 4);
         L.cnt = off; off += align_up((size_t)ceil_div(N, 32) * 4);
     }
@@ -157,6 +159,8 @@ int forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const floa
     g.Xo = at<__half>(ws, L.xo); g.Wo = at<__half>(ws, L.wo); g.kcap = L.kcap; g.n_outliers = &hdr->n_outliers;
     g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
     g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    g.sk_partial = at<int32_t>(ws, L.sk);
+    g.sk_flags = at<uint32_t>(ws, kWsSkFlagOffset);
     return from_cuda(launch_gemm_tc(g, s));
 }
 
@@ -301,6 +305,8 @@ int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t
     GemmArgs g{};
     g.CA = CA; g.CB = CB; g.C32 = C;
     g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    g.sk_partial = at<int32_t>(ws, L.sk);
+    g.sk_flags = at<uint32_t>(ws, kWsSkFlagOffset);
     return from_cuda(launch_gemm_tc(g, s));
 }
 

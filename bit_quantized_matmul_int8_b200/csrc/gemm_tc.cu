@@ -1,7 +1,7 @@
 // Prefill path of the LLM.int8() forward on sm_100a tensor cores.
 //
 // Computes, per 256 x 256 output tile,
-//     Y = fp16( C * SCA[i] * SCB[j] / 127^2 + P + bias[j] )
+//     Y = fp16( C * SCA[i] * SCB[j] / 127^2 + bias[j] + P )
 //     C = CA . CB^T    int8 x int8 -> int32   ("Int8 Matrix Multiplication with
 //                      16-bit Float Inputs and Outputs" and "Vector-wise
 //                      Quantization", LLM.int8() paper summary)
@@ -11,23 +11,23 @@
 // is computed by one pair with 2-SM tensor-core MMAs (tcgen05 cta_group::2):
 // each CTA stages its own 128 rows of A and its own half (128 rows) of B,
 // so per SM a 128 x 256 x 128 k-block needs 32 KB of operands instead of
-// 48 KB, and a 6-deep ring of stages fits in shared memory.
-//   warp 0     (both CTAs) TMA producer into a 6-stage ring; the loads of
-//              both CTAs complete on the leader CTA's full barrier;
-//   warp 1     (both CTAs) allocates the 512 tensor-memory columns; in the
-//              leader it issues the pair MMAs and multicasts the commits;
-//   warps 2-9  (both CTAs) epilogue on the CTA's 128 rows: tcgen05.ld the
-//              accumulator, dequantize in fp32, add P and bias, and store fp16
-//              through shared memory with TMA (32 x 32 boxes, double buffered
-//              per warp), so the epilogue warps never wait on global stores.
-// Outlier product, chosen on the device from |O| (no host sync):
-//   |O| <= kEpiOutlierMax: two int32 accumulators of 256 columns (double
-//       buffered: the epilogue of one tile overlaps the mainloop of the next)
-//       and P on the CUDA cores in the epilogue, from the row's Xo values in
-//       registers and the tile's Wo in shared memory; every fp16 x fp16
-//       product is exact in fp32, as on the tensor cores;
-//   |O| >  kEpiOutlierMax: one int32 accumulator (columns 0-255) and P as
-//       tcgen05 kind::f16 MMAs into an fp32 accumulator (columns 256-511).
+// 48 KB, and a 5-deep ring of stages fits in shared memory.
+//   warp 0     (both CTAs) TMA producer: the int8 k-blocks into the ring, and
+//              the tile's outlier columns (Xo, Wo: 32 fp16 per row, 64-byte
+//              swizzle) into a slot of their own; the loads of both CTAs
+//              complete on the leader CTA's barriers;
+//   warp 1     (both CTAs) allocates the 512 tensor-memory columns: two int32
+//              accumulators of 256 columns, so the epilogue of one tile
+//              overlaps the mainloop of the next; in the leader it issues the
+//              pair MMAs and multicasts the commits;
+//   warps 2-9  (both CTAs) epilogue on the CTA's 128 rows.
+// With outlier columns (|O| > 0) the epilogue runs in two passes over the
+// tile's accumulator: it dequantizes the int32 sums to fp32 (plus bias) and
+// writes them back into the same tensor-memory columns; the MMA warp then
+// adds P there with kind::f16 MMAs (fp32 accumulate, K = 16 per MMA) while
+// the next tile's int8 MMAs run; the second pass converts to fp16 and stores
+// through shared memory with TMA (32 x 32 boxes, double buffered per warp).
+// Without outliers the epilogue is a single pass.
 // Every wait is bounded (kWaitLimitNs); a wait that runs out sets the
 // workspace status word and the kernel winds down without touching Y.
 #include <algorithm>
@@ -37,6 +37,58 @@
 
 namespace int8lt {
 
+// Work of one CTA pair. Whole tiles round-robin over the pairs ("data
+// parallel"), and, when the tile count is not a multiple of the pair count,
+// the last one to two waves' worth of tiles are cut into k-block ranges of
+// equal length, one per pair ("stream-K"), so every pair gets the same
+// number of k-blocks. A range covers at least one tile, so a tile is split
+// at most once: its first k-blocks end pair p's range (the "head", which
+// finishes the tile) and its last k-blocks start pair p + 1's range (the
+// "tail", which hands its int32 partial sums over through global memory).
+struct Seg {
+    int tile, kb0, kb1;
+    bool head, tail;
+};
+
+struct TileSched {
+    int num_tiles, nkb, total_kb, num_pairs, pair, dp_tiles;
+    int64_t r, r_end;   // stream-K k-block cursor of this pair
+    int dp_next;
+
+    __host__ __device__ TileSched(int tiles, int nkb_, int total_kb_, int pairs, int p, bool sk_on)
+        : num_tiles(tiles), nkb(nkb_), total_kb(total_kb_), num_pairs(pairs), pair(p) {
+        dp_tiles = tiles;
+        r = r_end = 0;
+        if (sk_on && tiles > pairs && tiles % pairs != 0) {
+            const int full = tiles / pairs;
+            dp_tiles = (full - 1) * pairs;
+            const int64_t iters = (int64_t)(tiles - dp_tiles) * nkb;
+            r = iters * p / pairs;
+            r_end = iters * (p + 1) / pairs;
+        }
+        dp_next = p;
+    }
+    __host__ __device__ bool next(Seg &g) {
+        if (dp_next < dp_tiles) {
+            g.tile = dp_next;
+            g.kb0 = 0;
+            g.kb1 = total_kb;
+            g.head = g.tail = false;
+            dp_next += num_pairs;
+            return true;
+        }
+        if (r >= r_end) return false;
+        g.tile = dp_tiles + (int)(r / nkb);
+        g.kb0 = (int)(r % nkb);
+        const int64_t left = r_end - r;
+        g.kb1 = left < (int64_t)(nkb - g.kb0) ? g.kb0 + (int)left : nkb;
+        g.head = g.kb0 == 0 && g.kb1 < nkb;
+        g.tail = g.kb0 > 0;
+        r += g.kb1 - g.kb0;
+        return true;
+    }
+};
+
 namespace {
 
 constexpr int BM = 256, BN = 256;         // pair tile
@@ -45,11 +97,13 @@ constexpr int kStages = 5;
 constexpr int kStageA = kCtaRows * 128;   // bytes: 128 rows x 128 B
 constexpr int kStageB = kCtaRows * 128;   // bytes: 128 rows x 128 B (half of N)
 constexpr uint32_t kTxBytes = 2 * (kStageA + kStageB);  // both CTAs, counted by the leader
+constexpr int kOkb = 32;                  // outlier columns per k-block (64-byte rows)
+constexpr int kOStage = kCtaRows * kOkb * 2;            // bytes of Xo (or Wo) per CTA: 8 KB
+constexpr uint32_t kOTxBytes = 2 * 2 * kOStage;         // Xo + Wo of both CTAs
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kEpiOutlierMax = 24;  // largest |O| whose product runs on the CUDA cores
 constexpr int kEpiBarrier = 1;            // named barrier of the epilogue warps
 constexpr uint16_t kPairMask = 0x3;       // both CTAs of the cluster
 
@@ -65,7 +119,11 @@ constexpr uint32_t kIdescF16 = (1u << 4)     // D = f32, A = B = f16 (0)
 struct __align__(8) Ctrl {
     uint64_t full[kStages];     // leader: both CTAs' stage bytes landed
     uint64_t empty[kStages];    // each CTA: the pair MMAs are done with the stage
-    uint64_t acc_full[2];       // each CTA: the accumulator buffer is complete
+    uint64_t ofull;             // leader: both CTAs' outlier k-block landed
+    uint64_t oempty;            // each CTA: the P MMAs are done with the outlier slot
+    uint64_t acc_full[2];       // each CTA: the buffer holds the tile's int32 sums
+    uint64_t acc_mid[2];        // leader: both CTAs' epilogues wrote fp32 into the buffer
+    uint64_t acc_p[2];          // each CTA: P has been added to the buffer
     uint64_t acc_empty[2];      // leader: both CTAs' epilogues have read the buffer
     uint64_t drain;             // each CTA: every pair MMA has finished
     uint32_t tmem_base;
@@ -76,120 +134,121 @@ struct __align__(8) Ctrl {
 constexpr int kStoreBox = 32;                                    // Y staged in 32 x 32 fp16 boxes
 constexpr size_t kStoreBufBytes = kStoreBox * kStoreBox * 2;     // 2 KB
 constexpr size_t kSmemTiles = (size_t)kStages * (kStageA + kStageB);
-constexpr size_t kOffStage = kSmemTiles;                         // [kEpiWarps][2] store boxes
+constexpr size_t kOffOut = kSmemTiles;                           // Xo slot, then Wo slot
+constexpr size_t kOffStage = kOffOut + 2 * (size_t)kOStage;      // [kEpiWarps][2] store boxes
 constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * 2 * kStoreBufBytes;
 constexpr size_t kOffScb = kOffCtrl + 256;
 constexpr size_t kOffBias = kOffScb + BN * 4;
-constexpr size_t kOffWo = kOffBias + BN * 4;                     // fp32 [kEpiOutlierMax][BN]
-constexpr size_t kSmemUsed = kOffWo + (size_t)kEpiOutlierMax * BN * 4;
+constexpr size_t kSmemUsed = kOffBias + BN * 4;
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kSmemUsed;
 static_assert(sizeof(Ctrl) <= 256, "control block");
+static_assert(kOffOut % 1024 == 0 && kOStage % 1024 == 0, "swizzle atoms need aligned slots");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync %0, %1;" ::"r"(kEpiBarrier), "r"(kEpiThreads) : "memory");
 }
 
-// Epilogue of one tile for one warp: 32 rows (TMEM lanes) x 128 columns, in
-// chunks of 32. kMmaOut: the outlier product P is in TMEM (fp32, 256 columns
-// after the int32 sums); otherwise it is computed here from Xo and Wo.
-template <bool kMmaOut>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs &a, uint32_t tmem, uint32_t lane_base, int buf, int hcol,
-                                              int q, int lane, int ew, uint32_t rank, bool row_ok, int64_t row,
-                                              float rs, int64_t n0, int64_t m0, int n_out, const float *s_scb,
-                                              const float *s_bias, const float *s_wo, uint8_t *s_stage, int &sbuf,
-                                              Ctrl *ctrl, const CUtensorMap *tmY,
-                                              const uint4 (&xo_v)[kEpiOutlierMax / 8]) {
-    const bool cuda_out = !kMmaOut && n_out > 0;
-    // This row's outlier activations (CUDA-core outlier product), fp16.
-    const __half *xo = reinterpret_cast<const __half *>(xo_v);
+__device__ __forceinline__ uint32_t ld_acquire_flag(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Hand a TMEM buffer back to the leader's MMA warp (or signal the leader's
+// acc_mid barrier): one arrival per epilogue warp of each CTA.
+__device__ __forceinline__ void arrive_leader(Ctrl *ctrl, uint64_t *bar, uint32_t rank) {
+    const uint32_t b = smem_u32(bar);
+    if (rank == 0) mbar_arrive(b); else mbar_arrive_cluster(mapa_shared(b, 0));
+}
+
+// Partial sums of a split tile's tail, written so that each store of a
+// warp covers 512 contiguous bytes: int4 (v) of chunk cc of lane l of
+// epilogue warp ew sits at slot[((ew * 4 + cc / 32) * 8 + v) * 32 + l]. The
+// head reads them back with the same warp and lane, which own the same rows
+// and columns in both CTAs' epilogues.
+__device__ __forceinline__ void epilogue_store_partial(uint32_t tmem, uint32_t lane_base, int buf, int hcol, int ew,
+                                                       int lane, uint32_t rank, Ctrl *ctrl, int4 *slot) {
     const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
+    int4 *dst = slot + (size_t)ew * 4 * 8 * 32 + lane;
     for (int cc = 0; cc < 128; cc += 32) {
-        const int c = hcol * 128 + cc;  // column within the tile
-        uint32_t acc[32], po[32];
+        uint32_t acc[32];
         tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
-        if constexpr (kMmaOut) tmem_ld_32x32b_x32(tmem + lane_base + 256 + col0 + cc, po);
         tmem_ld_wait();
         if (cc == 96) {
-            // Every TMEM read of this buffer is done: hand it back to
-            // the leader's MMA warp.
             tc_fence_before();
-            if (lane == 0) {
-                const uint32_t eb = smem_u32(&ctrl->acc_empty[buf]);
-                if (rank == 0) mbar_arrive(eb); else mbar_arrive_cluster(mapa_shared(eb, 0));
-            }
+            if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
         }
-        if (n0 + c >= a.N) continue;  // whole chunk past the last column
-        if (a.C32) {
-            if (!row_ok) continue;
-            int32_t *dst = a.C32 + row * a.N + n0 + c;
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-                if (n0 + c + 4 * v < a.N)
-                    reinterpret_cast<int4 *>(dst)[v] =
-                        make_int4((int)acc[4 * v], (int)acc[4 * v + 1], (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
-            continue;
-        }
-        // y = C * SCA / 127^2 * SCB + bias (+ P), two columns per
-        // packed fp32x2 operation (each lane rounds like fmaf/fmul).
-        float2 y2[16];
-        const float2 rs2 = make_float2(rs, rs);
-        const float4 *sc4 = reinterpret_cast<const float4 *>(s_scb + c);
-        const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias + c);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const float4 sc = sc4[v], bi = bi4[v];
-            const float2 c01 = __fmul2_rn(make_float2((float)(int32_t)acc[4 * v], (float)(int32_t)acc[4 * v + 1]), rs2);
-            const float2 c23 =
-                __fmul2_rn(make_float2((float)(int32_t)acc[4 * v + 2], (float)(int32_t)acc[4 * v + 3]), rs2);
-            y2[2 * v] = __ffma2_rn(c01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
-            y2[2 * v + 1] = __ffma2_rn(c23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
-        }
-        if constexpr (kMmaOut) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                y2[k] = __fadd2_rn(y2[k], make_float2(__uint_as_float(po[2 * k]), __uint_as_float(po[2 * k + 1])));
-        }
-        if (!kMmaOut && cuda_out) {
-#pragma unroll
-            for (int t = 0; t < (kMmaOut ? 1 : kEpiOutlierMax); ++t) {
-                if (t >= n_out) break;  // uniform across the CTA
-                const float xt = __half2float(xo[t]);
-                const float2 xv = make_float2(xt, xt);
-                const float4 *w4 = reinterpret_cast<const float4 *>(s_wo + t * BN + c);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 wv = w4[v];
-                    y2[2 * v] = __ffma2_rn(xv, make_float2(wv.x, wv.y), y2[2 * v]);
-                    y2[2 * v + 1] = __ffma2_rn(xv, make_float2(wv.z, wv.w), y2[2 * v + 1]);
-                }
-            }
-        }
-        uint32_t packed[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            __half2 h = __float22half2_rn(y2[k]);
-            packed[k] = *reinterpret_cast<uint32_t *>(&h);
-        }
-        // Stage the warp's 32 x 32 box in shared memory (64-byte swizzle:
-        // 16-byte chunk i of row r sits at chunk i ^ ((r >> 1) & 3), which
-        // keeps the four stores of each row conflict-free) and hand it to
-        // the TMA engine. Rows and columns past M and N are clipped by it.
-        if (lane == 0) bulk_wait_read_1();  // this buffer's previous store has read it
-        __syncwarp();
-        uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
-                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d(tmY, smem_u32(box), (int32_t)(n0 + c), (int32_t)(m0 + q * 32));
-            bulk_commit_group();
-        }
-        sbuf ^= 1;
+        for (int v = 0; v < 8; ++v)
+            __stcg(dst + ((cc >> 5) * 8 + v) * 32,
+                   make_int4((int)acc[4 * v], (int)acc[4 * v + 1], (int)acc[4 * v + 2], (int)acc[4 * v + 3]));
     }
+}
+
+// Head of a split tile: add the tail's int32 sums of this warp's chunk cc
+// (exact), read in the layout epilogue_store_partial wrote.
+__device__ __forceinline__ void add_partial(uint32_t (&acc)[32], const int4 *part, int cc) {
+    if (!part) return;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const int4 t = __ldcg(part + ((cc >> 5) * 8 + v) * 32);
+        acc[4 * v] += (uint32_t)t.x;
+        acc[4 * v + 1] += (uint32_t)t.y;
+        acc[4 * v + 2] += (uint32_t)t.z;
+        acc[4 * v + 3] += (uint32_t)t.w;
+    }
+}
+
+// acc (int32 sums of 32 columns, plus the tail's partial sums if any) ->
+// fp32 C * rs * SCB[j] + bias[j], in place as bit patterns, two columns per
+// packed fp32x2 operation (each lane rounds like fmaf/fmul).
+__device__ __forceinline__ void dequant32(uint32_t (&acc)[32], float rs, const float *s_scb, const float *s_bias,
+                                          const int4 *part, int cc) {
+    add_partial(acc, part, cc);
+    const float2 rs2 = make_float2(rs, rs);
+    const float4 *sc4 = reinterpret_cast<const float4 *>(s_scb);
+    const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const float4 sc = sc4[v], bi = bi4[v];
+        const float2 c01 = __fmul2_rn(make_float2((float)(int32_t)acc[4 * v], (float)(int32_t)acc[4 * v + 1]), rs2);
+        const float2 c23 = __fmul2_rn(make_float2((float)(int32_t)acc[4 * v + 2], (float)(int32_t)acc[4 * v + 3]), rs2);
+        const float2 y01 = __ffma2_rn(c01, make_float2(sc.x, sc.y), make_float2(bi.x, bi.y));
+        const float2 y23 = __ffma2_rn(c23, make_float2(sc.z, sc.w), make_float2(bi.z, bi.w));
+        acc[4 * v] = __float_as_uint(y01.x);
+        acc[4 * v + 1] = __float_as_uint(y01.y);
+        acc[4 * v + 2] = __float_as_uint(y23.x);
+        acc[4 * v + 3] = __float_as_uint(y23.y);
+    }
+}
+
+// fp32 (bit patterns) -> fp16, staged in the warp's next 32 x 32 box in shared
+// memory (64-byte swizzle: 16-byte chunk i of row r sits at chunk
+// i ^ ((r >> 1) & 3), which keeps the four stores of each row conflict-free)
+// and handed to the TMA engine. Rows and columns past M and N are clipped by it.
+__device__ __forceinline__ void store32(const uint32_t (&y)[32], uint8_t *s_stage, int ew, int &sbuf, int lane,
+                                        const CUtensorMap *tmY, int32_t x, int32_t yrow) {
+    uint32_t packed[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        __half2 h = __float22half2_rn(make_float2(__uint_as_float(y[2 * k]), __uint_as_float(y[2 * k + 1])));
+        packed[k] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    if (lane == 0) bulk_wait_read_1();  // this box's previous store has read it
+    __syncwarp();
+    uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
+            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmY, smem_u32(box), x, yrow);
+        bulk_commit_group();
+    }
+    sbuf ^= 1;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -201,30 +260,33 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + kStages * kStageA;
+    uint8_t *sXo = smem + kOffOut;
+    uint8_t *sWo = smem + kOffOut + kOStage;
     Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem + kOffCtrl);
     float *s_scb = reinterpret_cast<float *>(smem + kOffScb);
     float *s_bias = reinterpret_cast<float *>(smem + kOffBias);
-    float *s_wo = reinterpret_cast<float *>(smem + kOffWo);
     uint8_t *s_stage = smem + kOffStage;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();          // 0: leader, 1: follower
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int nkb = (int)ceil_div(a.K, 128);
-    const int n_out = a.n_outliers ? *a.n_outliers : 0;
-    const bool mma_out = n_out > kEpiOutlierMax;       // outlier product on the tensor cores
-    const int nbuf = mma_out ? 1 : 2;                  // accumulator buffers in TMEM
-    const int n_mma_o = mma_out ? (n_out + 15) >> 4 : 0;   // fp16 MMAs of K = 16
-    const int nkb_o = mma_out ? (n_out + 63) >> 6 : 0;     // fp16 k-blocks of 64
-    const int total_kb = nkb + nkb_o;
+    const int n_out = (a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
+    const int n_okb = (n_out + kOkb - 1) / kOkb;       // outlier k-blocks per tile
+    const int n_mma_o = (n_out + 15) >> 4;             // fp16 MMAs of K = 16 per tile
+    const bool sk_on = a.sk_partial && a.sk_flags && num_pairs <= kSkMaxPairs;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&ctrl->full[s]), 1);
             mbar_init(smem_u32(&ctrl->empty[s]), 1);
         }
+        mbar_init(smem_u32(&ctrl->ofull), 1);
+        mbar_init(smem_u32(&ctrl->oempty), 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctrl->acc_full[b]), 1);
+            mbar_init(smem_u32(&ctrl->acc_mid[b]), 2 * kEpiWarps);
+            mbar_init(smem_u32(&ctrl->acc_p[b]), 1);
             mbar_init(smem_u32(&ctrl->acc_empty[b]), 2 * kEpiWarps);
         }
         mbar_init(smem_u32(&ctrl->drain), 1);
@@ -237,7 +299,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
         if (!a.C32) tma_prefetch(&tmY);
-        if (mma_out) {
+        if (n_okb) {
             tma_prefetch(&tmXo);
             tma_prefetch(&tmWo);
         }
@@ -259,33 +321,88 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
-            for (int tile = pair; tile < num_tiles && !*abort_flag; tile += num_pairs) {
-                const int32_t m0 = (tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
-                const int32_t n0 = (tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
-                for (int kb = 0; kb < total_kb; ++kb) {
+            // Outlier k-blocks go out in schedule order, for every segment
+            // that finishes a tile (not for tails), once the segment's int8
+            // k-blocks are all issued and the slot is free; waiting for a
+            // ring stage never blocks them.
+            TileSched tsp(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
+            Seg gp;
+            int p_avail = 0, p_done = 0, okb = 0;
+            bool have_gp = false;
+            uint32_t o_issued = 0;
+            auto pump = [&](bool block) {
+                while (p_done < p_avail && !*abort_flag) {
+                    if (!have_gp) {
+                        do { have_gp = tsp.next(gp); } while (have_gp && gp.tail);
+                        if (!have_gp) return;
+                    }
+                    const uint32_t eb = smem_u32(&ctrl->oempty);
+                    const uint32_t par = (o_issued & 1u) ^ 1u;
+                    if (block) {
+                        if (!mbar_wait_bounded(eb, par, kWaitLimitNs)) {
+                            *abort_flag = 1;
+                            record_timeout(a.status);
+                            return;
+                        }
+                    } else if (!mbar_try_wait(eb, par)) {
+                        return;
+                    }
+                    const uint32_t fb = smem_u32(&ctrl->ofull);
+                    if (rank == 0) mbar_arrive_expect_tx(fb, kOTxBytes);
+                    const uint32_t fb_leader = mapa_shared(fb, 0);
+                    const int32_t m0 = (gp.tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
+                    const int32_t n0 = (gp.tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
+                    tma_load_2d_pair(smem_u32(sXo), &tmXo, fb_leader, okb * kOkb, m0);
+                    tma_load_2d_pair(smem_u32(sWo), &tmWo, fb_leader, okb * kOkb, n0);
+                    ++o_issued;
+                    if (++okb == n_okb) {
+                        okb = 0;
+                        ++p_done;
+                        have_gp = false;
+                    }
+                }
+            };
+            TileSched ts(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
+            Seg g;
+            while (!*abort_flag && ts.next(g)) {
+                const int32_t m0 = (g.tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
+                const int32_t n0 = (g.tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
+                for (int kb = g.kb0; kb < g.kb1; ++kb) {
                     if (*abort_flag) break;
-                    if (!mbar_wait_bounded(smem_u32(&ctrl->empty[stage]), phase ^ 1u, kWaitLimitNs)) {
-                        *abort_flag = 1;
-                        record_timeout(a.status);
-                        break;
+                    const uint32_t eb = smem_u32(&ctrl->empty[stage]);
+                    if (!mbar_try_wait(eb, phase ^ 1u)) {
+                        const uint64_t t0 = globaltimer_ns();
+                        bool ok = true;
+                        while (!mbar_try_wait(eb, phase ^ 1u)) {
+                            if (n_okb) pump(false);
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!ok) {
+                            *abort_flag = 1;
+                            record_timeout(a.status);
+                            break;
+                        }
                     }
                     const uint32_t fb = smem_u32(&ctrl->full[stage]);
                     if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
                     const uint32_t fb_leader = mapa_shared(fb, 0);
-                    if (kb < nkb) {
-                        tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmA, fb_leader, kb * 128, m0);
-                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmB, fb_leader, kb * 128, n0);
-                    } else {
-                        const int ko = (kb - nkb) * 64;
-                        tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmXo, fb_leader, ko, m0);
-                        tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmWo, fb_leader, ko, n0);
-                    }
+                    tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmA, fb_leader, kb * 128, m0);
+                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmB, fb_leader, kb * 128, n0);
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
+                if (n_okb && !g.tail) {
+                    ++p_avail;
+                    pump(false);
+                }
             }
+            if (n_okb) pump(true);
             // Do not leave while copies this thread started are in flight:
-            // a stage is free again once the pair MMAs have consumed it.
+            // a stage (or the outlier slot) is free again once the pair MMAs
+            // have consumed it.
             for (int u = max(0, issued - kStages); u < issued; ++u) {
                 const int s = u % kStages;
                 if (!mbar_wait_bounded(smem_u32(&ctrl->empty[s]), (uint32_t)((u / kStages) & 1), kWaitLimitNs)) {
@@ -293,16 +410,60 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     break;
                 }
             }
+            if (o_issued && !mbar_wait_bounded(smem_u32(&ctrl->oempty), (o_issued - 1u) & 1u, kWaitLimitNs))
+                record_timeout(a.status);
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ----------------------------------------- MMA issuer (leader) --
             int stage = 0;
             uint32_t phase = 0;
-            int it = 0;  // local tile count
-            for (int tile = pair; tile < num_tiles && !*abort_flag; tile += num_pairs, ++it) {
-                const int buf = it % nbuf;
-                const uint32_t use = (uint32_t)(it / nbuf);
+            int it = 0;  // local segment count
+            uint32_t p_uses[2] = {0u, 0u};  // P passes per buffer so far
+            uint32_t o_used = 0;            // outlier k-blocks consumed so far
+            bool pend = false;              // a finished tile still waits for its P
+            int pbuf = 0;
+            // P of the pending tile: once both epilogues have written its fp32
+            // values into the buffer, accumulate Xo . Wo^T onto them.
+            auto issue_p = [&](bool block) {
+                const uint32_t mb = smem_u32(&ctrl->acc_mid[pbuf]);
+                const uint32_t par = p_uses[pbuf] & 1u;
+                if (block) {
+                    if (!mbar_wait_bounded(mb, par, kWaitLimitNs)) {
+                        *abort_flag = 1;
+                        record_timeout(a.status);
+                        pend = false;
+                        return;
+                    }
+                } else if (!mbar_try_wait(mb, par)) {
+                    return;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(pbuf * 256);
+                for (int j = 0; j < n_okb; ++j) {
+                    if (!mbar_wait_bounded(smem_u32(&ctrl->ofull), o_used & 1u, kWaitLimitNs)) {
+                        *abort_flag = 1;
+                        record_timeout(a.status);
+                        pend = false;
+                        return;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sdesc_k_sw64(smem_u32(sXo));
+                    const uint64_t db = sdesc_k_sw64(smem_u32(sWo));
+                    for (int k = 0; k < 2 && 2 * j + k < n_mma_o; ++k)  // K = 16 fp16 = 32 bytes each
+                        mma_f16_pair(d, da + 2 * k, db + 2 * k, kIdescF16, 1u);
+                    mma_commit_pair(smem_u32(&ctrl->oempty), kPairMask);
+                    ++o_used;
+                }
+                mma_commit_pair(smem_u32(&ctrl->acc_p[pbuf]), kPairMask);
+                ++p_uses[pbuf];
+                pend = false;
+            };
+            TileSched ts(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
+            Seg g;
+            for (; !*abort_flag && ts.next(g); ++it) {
+                const int buf = it & 1;
+                const uint32_t use = (uint32_t)(it >> 1);
                 if (!mbar_wait_bounded(smem_u32(&ctrl->acc_empty[buf]), (use & 1u) ^ 1u, kWaitLimitNs)) {
                     *abort_flag = 1;
                     record_timeout(a.status);
@@ -310,8 +471,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 tc_fence_after();
                 const uint32_t d_i32 = tmem + (uint32_t)(buf * 256);
-                const uint32_t d_f32 = tmem + 256;
-                for (int kb = 0; kb < total_kb; ++kb) {
+                for (int kb = g.kb0; kb < g.kb1; ++kb) {
                     if (*abort_flag) break;
                     if (!mbar_wait_bounded(smem_u32(&ctrl->full[stage]), phase, kWaitLimitNs)) {
                         *abort_flag = 1;
@@ -321,22 +481,22 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     tc_fence_after();
                     const uint64_t da = sdesc_k_sw128(smem_u32(sA + stage * kStageA));
                     const uint64_t db = sdesc_k_sw128(smem_u32(sB + stage * kStageB));
-                    if (kb < nkb) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)  // 4 x (K = 32 int8 = 32 bytes)
-                            mma_i8_pair(d_i32, da + 2 * k, db + 2 * k, kIdescI8, (kb | k) != 0);
-                    } else {
-                        const int kbo = kb - nkb;
-                        const int nk = min(4, n_mma_o - kbo * 4);
-                        for (int k = 0; k < nk; ++k)  // K = 16 fp16 = 32 bytes each
-                            mma_f16_pair(d_f32, da + 2 * k, db + 2 * k, kIdescF16, (kbo | k) != 0);
-                    }
+                    for (int k = 0; k < 4; ++k)  // 4 x (K = 32 int8 = 32 bytes)
+                        mma_i8_pair(d_i32, da + 2 * k, db + 2 * k, kIdescI8, (kb != g.kb0) || (k != 0));
                     mma_commit_pair(smem_u32(&ctrl->empty[stage]), kPairMask);
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (pend) issue_p(false);
                 }
-                // lands in both CTAs when this tile's MMAs are done
+                // lands in both CTAs when this segment's MMAs are done
                 mma_commit_pair(smem_u32(&ctrl->acc_full[buf]), kPairMask);
+                if (pend && !*abort_flag) issue_p(true);
+                if (n_okb && !g.tail) {
+                    pend = true;
+                    pbuf = buf;
+                }
             }
+            if (pend && !*abort_flag) issue_p(true);
             // Nothing may still write either CTA's TMEM when it is freed.
             mma_commit_pair(smem_u32(&ctrl->drain), kPairMask);
         }
@@ -350,17 +510,18 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int hcol = ew >> 2;                // columns [128 hcol, 128 hcol + 128)
         const int et = threadIdx.x - 64;         // 0..255
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const bool cuda_out = !mma_out && n_out > 0;
         int sbuf = 0;  // which of the warp's two store boxes is next
         int it = 0;
-        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++it) {
-            const int64_t m0 = (int64_t)(tile % num_m_tiles) * BM + rank * kCtaRows;
-            const int64_t n0 = (int64_t)(tile / num_m_tiles) * BN;
-            const int buf = it % nbuf;
-            const uint32_t use = (uint32_t)(it / nbuf);
+        uint32_t p_uses[2] = {0u, 0u};
+        TileSched ts(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
+        Seg g;
+        for (; ts.next(g); ++it) {
+            const int64_t m0 = (int64_t)(g.tile % num_m_tiles) * BM + rank * kCtaRows;
+            const int64_t n0 = (int64_t)(g.tile / num_m_tiles) * BN;
+            const int buf = it & 1;
+            const uint32_t use = (uint32_t)(it >> 1);
             // Fetch this tile's column data (thread et owns column n0 + et)
-            // and this thread's row data into registers while the MMAs are
-            // still running: 16-byte loads, all issued before any wait.
+            // and this thread's row scale while the MMAs are still running.
             const int64_t col = n0 + et;
             const bool col_ok = !a.C32 && col < a.N;
             const float scb_v = col_ok ? a.SCB[col] : 0.f;
@@ -368,15 +529,6 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int64_t row = m0 + q * 32 + lane;
             const bool row_ok = row < a.M;
             const float sca_v = (row_ok && a.SCA) ? a.SCA[row] : 0.f;
-            uint4 wo_v[kEpiOutlierMax / 8], xo_v[kEpiOutlierMax / 8];
-#pragma unroll
-            for (int v = 0; v < kEpiOutlierMax / 8; ++v) {
-                const bool need = cuda_out && 8 * v < n_out;
-                wo_v[v] = (need && col_ok) ? *reinterpret_cast<const uint4 *>(a.Wo + col * a.kcap + 8 * v)
-                                           : make_uint4(0, 0, 0, 0);
-                xo_v[v] = (need && row_ok) ? *reinterpret_cast<const uint4 *>(a.Xo + row * a.kcap + 8 * v)
-                                           : make_uint4(0, 0, 0, 0);
-            }
             // Wait for the accumulator, then decide together whether to go
             // on: every epilogue warp votes before the barrier and reads the
             // same slot after it, so all of them leave the loop together.
@@ -394,22 +546,115 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (!a.C32) {
                 s_scb[et] = scb_v;
                 s_bias[et] = bias_v;
-                if (cuda_out) {
-                    const __half *wh = reinterpret_cast<const __half *>(wo_v);
-#pragma unroll
-                    for (int t = 0; t < kEpiOutlierMax; ++t)
-                        if (t < n_out) s_wo[t * BN + et] = __half2float(wh[t]);
-                }
             }
             epi_sync();
             tc_fence_after();
+            const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
+            if (g.tail) {
+                // Tail of a split tile: hand the int32 sums to the head's pair.
+                int4 *slot = reinterpret_cast<int4 *>(a.sk_partial) + (size_t)(pair * 2 + rank) * (kSkPartialBytes / 16);
+                epilogue_store_partial(tmem, lane_base, buf, hcol, ew, lane, rank, ctrl, slot);
+                __threadfence();
+                epi_sync();
+                if (et == 0) atomicExch(&a.sk_flags[pair * 2 + rank], 1u);
+                continue;
+            }
+            const int4 *part = nullptr;
+            if (g.head) {
+                // Head of a split tile: the next pair wrote the tail's sums at
+                // the start of its range; wait (bounded) until they are visible.
+                const uint32_t *flag = &a.sk_flags[(pair + 1) * 2 + rank];
+                if (et == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_flag(flag) == 0) {
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            record_timeout(a.status);
+                            break;
+                        }
+                    }
+                }
+                epi_sync();
+                part = reinterpret_cast<const int4 *>(a.sk_partial) +
+                       (size_t)((pair + 1) * 2 + rank) * (kSkPartialBytes / 16) + (size_t)ew * 4 * 8 * 32 + lane;
+            }
             const float rs = sca_v * (1.0f / 16129.0f);
-            if (mma_out)
-                epilogue_tile<true>(a, tmem, lane_base, buf, hcol, q, lane, ew, rank, row_ok, row, rs, n0, m0, n_out,
-                                    s_scb, s_bias, s_wo, s_stage, sbuf, ctrl, &tmY, xo_v);
-            else
-                epilogue_tile<false>(a, tmem, lane_base, buf, hcol, q, lane, ew, rank, row_ok, row, rs, n0, m0, n_out,
-                                     s_scb, s_bias, s_wo, s_stage, sbuf, ctrl, &tmY, xo_v);
+            if (a.C32) {
+                // Raw int32 sums (test entry): no scales, no outliers.
+                for (int cc = 0; cc < 128; cc += 32) {
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+                    tmem_ld_wait();
+                    if (cc == 96) {
+                        tc_fence_before();
+                        if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
+                    }
+                    add_partial(acc, part, cc);
+                    const int64_t c0 = n0 + hcol * 128 + cc;
+                    if (!row_ok || c0 >= a.N) continue;
+                    int32_t *dst = a.C32 + row * a.N + c0;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        if (c0 + 4 * v < a.N)
+                            reinterpret_cast<int4 *>(dst)[v] = make_int4((int)acc[4 * v], (int)acc[4 * v + 1],
+                                                                         (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
+                }
+            } else if (n_okb) {
+                // Pass 1: fp32 C * rs * SCB + bias back into the buffer.
+                for (int cc = 0; cc < 128; cc += 32) {
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+                    tmem_ld_wait();
+                    dequant32(acc, rs, s_scb + hcol * 128 + cc, s_bias + hcol * 128 + cc, part, cc);
+                    tmem_st_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                if (lane == 0) arrive_leader(ctrl, &ctrl->acc_mid[buf], rank);
+                // The MMA warp adds P; all warps vote on the outcome together.
+                bool pok = mbar_wait_bounded(smem_u32(&ctrl->acc_p[buf]), p_uses[buf] & 1u, kWaitLimitNs);
+                if (!pok) record_timeout(a.status);
+                ++p_uses[buf];
+                pok = __all_sync(0xffffffffu, pok);
+                if (lane == 0 && !pok) *vote = 1;
+                epi_sync();
+                if (*vote) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                // Pass 2: fp16 out.
+                for (int cc = 0; cc < 128; cc += 32) {
+                    uint32_t y[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, y);
+                    tmem_ld_wait();
+                    if (cc == 96) {
+                        tc_fence_before();
+                        if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
+                    }
+                    if (n0 + hcol * 128 + cc < a.N)
+                        store32(y, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * 128 + cc),
+                                (int32_t)(m0 + q * 32));
+                }
+            } else {
+                // No outliers: one pass.
+                for (int cc = 0; cc < 128; cc += 32) {
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
+                    tmem_ld_wait();
+                    if (cc == 96) {
+                        tc_fence_before();
+                        if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
+                    }
+                    if (n0 + hcol * 128 + cc >= a.N) continue;  // whole chunk past the last column
+                    dequant32(acc, rs, s_scb + hcol * 128 + cc, s_bias + hcol * 128 + cc, part, cc);
+                    store32(acc, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * 128 + cc),
+                            (int32_t)(m0 + q * 32));
+                }
+            }
+            if (g.head) {
+                epi_sync();  // every warp has read the tail's sums
+                if (et == 0) a.sk_flags[(pair + 1) * 2 + rank] = 0u;
+            }
         }
         if (lane == 0) bulk_wait_all();  // every store of this warp has finished
     }
@@ -473,8 +718,10 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
         !make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CB, a.K, a.N, a.K, 128, kCtaRows))
         return cudaErrorInvalidValue;
     if (a.Xo && a.Wo && a.n_outliers) {
-        if (!make_map(&mXo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Xo, a.kcap, a.M, a.kcap * 2, 64, kCtaRows) ||
-            !make_map(&mWo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Wo, a.kcap, a.N, a.kcap * 2, 64, kCtaRows))
+        if (!make_map(&mXo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Xo, a.kcap, a.M, a.kcap * 2, kOkb, kCtaRows,
+                      CU_TENSOR_MAP_SWIZZLE_64B) ||
+            !make_map(&mWo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Wo, a.kcap, a.N, a.kcap * 2, kOkb, kCtaRows,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
             return cudaErrorInvalidValue;
     } else {
         mXo = mA;  // never read: |O| = 0 without outlier buffers
@@ -519,3 +766,22 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
 }
 
 }  // namespace int8lt
+
+// Test entry: the stream-K schedule as the GEMM walks it, enumerated on the
+// host. Rows of 6 int32: pair, tile, kb0, kb1, head, tail.
+extern "C" int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int32_t *out, int cap_rows) {
+    if (tiles < 0 || nkb < 1 || pairs < 1 || (!out && cap_rows > 0)) return -1;
+    int n = 0;
+    for (int p = 0; p < pairs; ++p) {
+        int8lt::TileSched ts(tiles, nkb, nkb, pairs, p, pairs <= int8lt::kSkMaxPairs);
+        int8lt::Seg g;
+        while (ts.next(g)) {
+            if (n < cap_rows) {
+                int32_t *r = out + 6 * n;
+                r[0] = p; r[1] = g.tile; r[2] = g.kb0; r[3] = g.kb1; r[4] = g.head; r[5] = g.tail;
+            }
+            ++n;
+        }
+    }
+    return n;
+}

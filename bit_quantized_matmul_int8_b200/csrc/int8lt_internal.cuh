@@ -29,7 +29,7 @@ struct WsLayout {
     int64_t M, N, K;
     int64_t kwords;        // ceil(K / 32): words of one column bitmap
     int64_t kcap;          // round_up(K, 64): row pitch (elements) of Xo / Wo
-    size_t hdr, bitmaps, idx, sca, ca, xo, wo, acc, cnt, total;
+    size_t hdr, bitmaps, idx, sca, ca, xo, wo, acc, cnt, sk, total;
 };
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K);
 
@@ -38,11 +38,18 @@ struct WsHeader {
     uint32_t status;       // kStatus* bits, sticky until read
     int32_t n_outliers;    // |O| of the last quantize pass
     uint32_t qgen;         // quantize launches so far: selects this launch's bitmap
-    uint32_t bar_count;    // arrivals at the quantize grid barrier (0 between launches)
-    uint32_t pad[60];
+    uint32_t bar_count;    // arrivals at the quantize grid barrier, all launches (wraps)
+    uint32_t qbase;        // bar_count when the next quantize launch starts
+    uint32_t pad[59];
 };
 constexpr size_t kWsBitmapOffset = 1024;
-constexpr size_t kWsInitBytes = kWsBitmapOffset + 2 * (size_t)kMaxKwords * 4;
+// Stream-K of the prefill GEMM: one ready flag per (CTA pair, rank) in the
+// zeroed region, and one int32 partial tile (128 x 256) per (pair, rank).
+constexpr int kSkMaxPairs = 80;
+constexpr size_t kSkPartialBytes = (size_t)128 * 256 * 4;
+constexpr size_t kWsSkFlagOffset = kWsBitmapOffset + ((2 * (size_t)kMaxKwords * 4 + 1023) & ~size_t(1023));
+constexpr size_t kWsInitBytes = kWsSkFlagOffset + 1024;
+static_assert(2 * kSkMaxPairs * 4 <= 1024, "stream-K flags");
 
 // ------------------------------------------------------------- launchers --
 
@@ -94,6 +101,9 @@ struct GemmArgs {
     int32_t *C32;             // debug: raw int32 output instead of Y
     int64_t M, N, K;
     uint32_t *status;
+    // Stream-K of the last wave (both null: whole tiles only).
+    int32_t *sk_partial;      // [kSkMaxPairs][2][128][256]
+    uint32_t *sk_flags;       // [kSkMaxPairs][2], zero between launches
 };
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 
@@ -272,6 +282,23 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Store 32 consecutive 32-bit TMEM columns of this warp's 32 lanes (one
+// lane per thread), the inverse of tmem_ld_32x32b_x32.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // 2-D tiled TMA store shared -> global (bulk-group completion). Elements of
 // the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src, int32_t x, int32_t y) {
@@ -374,6 +401,18 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
     d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset
     d |= (uint64_t)1 << 46;                    // descriptor version for tcgen05
     d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
+// Same for a K-major tile with 64-byte swizzling: rows of 64 bytes, 8-row
+// (512-byte) swizzle atoms stacked along M/N (stride byte offset 512).
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(512 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;                    // 64-byte swizzle
     return d;
 }
 

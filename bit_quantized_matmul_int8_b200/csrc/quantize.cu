@@ -62,10 +62,12 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+// Codes of the 8 fp16 values of a 16-byte vector (scalar fp32 multiply and
+// add per value, as code_bits()).
 __device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
     const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-    float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
-    float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
+    const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
+    const float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
     uint2 r;
     r.x = pack4(code_bits(f0.x, s), code_bits(f0.y, s), code_bits(f1.x, s), code_bits(f1.y, s));
     r.y = pack4(code_bits(f2.x, s), code_bits(f2.y, s), code_bits(f3.x, s), code_bits(f3.y, s));
@@ -158,12 +160,24 @@ __device__ __forceinline__ int64_t outlier_column(const uint32_t *bits, const in
 }
 
 // Outlier mask (bit j = column 8v + j) of the 16-byte vector v.
-__device__ __forceinline__ uint32_t vec_mask(const uint32_t *bits, int64_t v) {
-    return (bits[(v * 8) >> 5] >> ((v * 8) & 31)) & 0xffu;
+__device__ __forceinline__ uint32_t vec_mask(const uint32_t *bits, int v) {
+    return (bits[v >> 2] >> ((v & 3) * 8)) & 0xffu;
 }
 
 // Slow paths for the few vectors holding outlier columns, kept out of line
 // so the unrolled fast path does not reserve registers for them.
+// Phase A test of one vector of 8 halves: set bit (v*8 + k) of `bits` for
+// every element k with |x| >= threshold (t2 = the threshold's binary16 bits,
+// twice). A vector with no hit, the usual case, costs four compares.
+__device__ __forceinline__ void flag_vec(uint4 x, uint32_t t2, int v, uint32_t *bits) {
+    const uint32_t h0 = __vcmpgeu2(x.x & 0x7fff7fffu, t2), h1 = __vcmpgeu2(x.y & 0x7fff7fffu, t2);
+    const uint32_t h2 = __vcmpgeu2(x.z & 0x7fff7fffu, t2), h3 = __vcmpgeu2(x.w & 0x7fff7fffu, t2);
+    if ((h0 | h1 | h2 | h3) == 0u) return;
+    const uint32_t b = (h0 & 1u) | ((h0 >> 15) & 2u) | ((h1 & 1u) << 2) | ((h1 >> 13) & 8u) | ((h2 & 1u) << 4) |
+                       ((h2 >> 11) & 32u) | ((h3 & 1u) << 6) | ((h3 >> 9) & 128u);
+    atomicOr(&bits[v >> 2], b << ((v & 3) * 8));
+}
+
 __device__ __noinline__ uint32_t masked_absmax_bits_slow(uint4 x, uint32_t m) {
     const uint16_t *e = reinterpret_cast<const uint16_t *>(&x);
     uint32_t amax = 0;
@@ -178,7 +192,7 @@ __device__ __forceinline__ uint32_t masked_absmax_bits(uint4 x, uint32_t m) {
 }
 
 // Codes of vector v (outlier columns -> 0, and their fp16 values -> Xo).
-__device__ __noinline__ uint2 quant_masked_slow(uint4 x, uint32_t m, float s, int64_t v, const uint32_t *bits,
+__device__ __noinline__ uint2 quant_masked_slow(uint4 x, uint32_t m, float s, int v, const uint32_t *bits,
                                                 const int32_t *prefix, __half *xo) {
     uint2 q = quant_vec8(x, s);
     {
@@ -188,7 +202,7 @@ __device__ __noinline__ uint2 quant_masked_slow(uint4 x, uint32_t m, float s, in
         for (int j = 0; j < 8; ++j) {
             if ((m >> j) & 1u) {
                 if (xo) {
-                    const int64_t col = v * 8 + j;
+                    const int col = v * 8 + j;
                     const int32_t rank = prefix[col >> 5] + __popc(bits[col >> 5] & ((1u << (col & 31)) - 1u));
                     xo[rank] = e[j];
                 }
@@ -202,7 +216,7 @@ __device__ __noinline__ uint2 quant_masked_slow(uint4 x, uint32_t m, float s, in
     return q;
 }
 
-__device__ __forceinline__ uint2 quant_masked(uint4 x, uint32_t m, float s, int64_t v, const uint32_t *bits,
+__device__ __forceinline__ uint2 quant_masked(uint4 x, uint32_t m, float s, int v, const uint32_t *bits,
                                               const int32_t *prefix, __half *xo) {
     return m == 0 ? quant_vec8(x, s) : quant_masked_slow(x, m, s, v, bits, prefix, xo);
 }
@@ -231,13 +245,16 @@ template <int T, int V>
 __device__ __forceinline__ void quantize_row_regs(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
                                                   int32_t n_out, const uint4 (&x)[V], int64_t r, bool valid,
                                                   uint32_t *red, int team, int tl) {
-    const int64_t nvec = a.K / 8;
+    const int nvec = (int)(a.K / 8);
     const int32_t n16 = (n_out + 15) & ~15;
+    uint32_t m[V];
     uint32_t amax = 0;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-        const int64_t v = tl + (int64_t)i * T;
-        if (valid && v < nvec) amax = max(amax, masked_absmax_bits(x[i], vec_mask(bits, v)));
+        const int v = tl + i * T;
+        const bool in = valid && v < nvec;
+        m[i] = in ? vec_mask(bits, v) : 0u;
+        if (in) amax = max(amax, masked_absmax_bits(x[i], m[i]));
     }
     amax = team_max<T>(amax, red, team);
     if (!valid) return;
@@ -247,68 +264,55 @@ __device__ __forceinline__ void quantize_row_regs(const QuantizeArgs &a, const u
     __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-        const int64_t v = tl + (int64_t)i * T;
-        if (v < nvec) ca2[v] = quant_masked(x[i], vec_mask(bits, v), s, v, bits, prefix, xo);
+        const int v = tl + i * T;
+        if (v < nvec) ca2[v] = quant_masked(x[i], m[i], s, v, bits, prefix, xo);
     }
     if (xo)
         for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
     if (tl == 0) a.SCA[r] = sa;
 }
 
+// Load the V vectors of row r a team thread owns (zeros past the row end).
+template <int T, int V>
+__device__ __forceinline__ void load_row(const QuantizeArgs &a, int64_t r, int tl, uint4 (&x)[V]) {
+    const int nvec = (int)(a.K / 8);
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int v = tl + i * T;
+        x[i] = v < nvec ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// Phase B for the team's rows, re-read from memory (rows are not kept).
 template <int T, int V>
 __device__ void quantize_rows_team(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
                                    int32_t n_out, int row_ctas, uint32_t *red) {
     const int teams = kThreads / T;
     const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
-    const int64_t nvec = a.K / 8;
-    const int32_t n16 = (n_out + 15) & ~15;
     for (int64_t r = (int64_t)blockIdx.x * teams + team; r < a.M; r += (int64_t)row_ctas * teams) {
-        const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
-        uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
-        __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
-        uint32_t amax = 0;
-        float sa, s;
         if constexpr (V > 0) {
             uint4 x[V];
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                x[i] = v < nvec ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                if (v < nvec) amax = max(amax, masked_absmax_bits(x[i], vec_mask(bits, v)));
-            }
-            amax = team_max<T>(amax, red, team);
-            sa = __half2float(__ushort_as_half((unsigned short)amax));
-            s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                if (v < nvec) ca2[v] = quant_masked(x[i], vec_mask(bits, v), s, v, bits, prefix, xo);
-            }
+            load_row<T, V>(a, r, tl, x);
+            quantize_row_regs<T, V>(a, bits, prefix, n_out, x, r, true, red, team, tl);
         } else {
-            for (int64_t v = tl; v < nvec; v += T) amax = max(amax, masked_absmax_bits(__ldg(x4 + v), vec_mask(bits, v)));
+            const int nvec = (int)(a.K / 8);
+            const int32_t n16 = (n_out + 15) & ~15;
+            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
+            uint32_t amax = 0;
+            for (int v = tl; v < nvec; v += T) amax = max(amax, masked_absmax_bits(__ldg(x4 + v), vec_mask(bits, v)));
             amax = team_max<T>(amax, red, team);
-            sa = __half2float(__ushort_as_half((unsigned short)amax));
-            s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
-            for (int64_t v = tl; v < nvec; v += T)
+            const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+            const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+            uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+            __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
+            for (int v = tl; v < nvec; v += T)
                 ca2[v] = quant_masked(__ldg(x4 + v), vec_mask(bits, v), s, v, bits, prefix, xo);
+            if (xo)
+                for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
+            if (tl == 0) a.SCA[r] = sa;
         }
-        if (xo)
-            for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
-        if (tl == 0) a.SCA[r] = sa;
     }
-}
-
-// Outlier byte of a 16-byte vector: bit j set where |x_j| >= threshold,
-// decided on the fp16 magnitude bits against the threshold pattern.
-__device__ __forceinline__ uint32_t outlier_byte(uint4 v, uint32_t t2) {
-    const uint32_t h0 = __vcmpgeu2(v.x & 0x7fff7fffu, t2), h1 = __vcmpgeu2(v.y & 0x7fff7fffu, t2);
-    const uint32_t h2 = __vcmpgeu2(v.z & 0x7fff7fffu, t2), h3 = __vcmpgeu2(v.w & 0x7fff7fffu, t2);
-    return (h0 & 1u) | ((h0 >> 15) & 2u) | ((h1 & 1u) << 2) | ((h1 >> 13) & 8u) | ((h2 & 1u) << 4) |
-           ((h2 >> 11) & 32u) | ((h3 & 1u) << 6) | ((h3 >> 9) & 128u);
 }
 
 // Phase A for one team's rows: OR the rows' outlier bits into the CTA bitmap.
@@ -316,28 +320,20 @@ template <int T, int V>
 __device__ void flag_rows_team(const QuantizeArgs &a, uint32_t *bits, int teams_total) {
     const int teams = kThreads / T;
     const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
-    const int64_t nvec = a.K / 8;
+    const int nvec = (int)(a.K / 8);
     const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
     for (int64_t r = (int64_t)blockIdx.x * teams + team; r < a.M; r += teams_total) {
-        const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
         if constexpr (V > 0) {
             uint4 x[V];
+            load_row<T, V>(a, r, tl, x);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                x[i] = v < nvec ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                const uint32_t b = v < nvec ? outlier_byte(x[i], t2) : 0u;
-                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
+                const int v = tl + i * T;
+                if (v < nvec) flag_vec(x[i], t2, v, bits);
             }
         } else {
-            for (int64_t v = tl; v < nvec; v += T) {
-                const uint32_t b = outlier_byte(__ldg(x4 + v), t2);
-                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
-            }
+            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
+            for (int v = tl; v < nvec; v += T) flag_vec(__ldg(x4 + v), t2, v, bits);
         }
     }
 }
@@ -348,24 +344,27 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
     return v;
 }
 
-// Grid-wide barrier of the cooperative launch. The last CTA to arrive resets
-// the count and advances the generation, which releases the others; every
-// wait is bounded. Returns false (and records a timeout) if it ran out.
-__device__ bool grid_barrier(WsHeader *h, uint32_t gen) {
+// Grid-wide barrier of the cooperative launch. The arrival count only grows:
+// this launch's CTAs are all in once it reaches base + gridDim.x, which the
+// waiters see directly in the count. The last CTA in publishes the next
+// launch's base and generation (no CTA of this launch reads them any more;
+// the next launch, behind this one in stream order, does). Every wait is
+// bounded; after a timeout the count is off and the workspace header must be
+// initialised again. Returns false (and records a timeout) if it ran out.
+__device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base) {
     __shared__ uint32_t s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t ok = 1;
+        const uint32_t target = base + gridDim.x;
         __threadfence();
         const uint32_t old = atomicAdd(&h->bar_count, 1u);
-        if (old == gridDim.x - 1) {
-            // Release the waiters first; the count is reset for the next
-            // launch, which stream order keeps behind this one.
+        if (old == target - 1u) {
+            *reinterpret_cast<volatile uint32_t *>(&h->qbase) = target;
             atomicExch(&h->qgen, gen + 1u);
-            atomicExch(&h->bar_count, 0u);
         } else {
             const uint64_t t0 = globaltimer_ns();
-            while (ld_acquire_u32(&h->qgen) == gen) {
+            while ((int32_t)(ld_acquire_u32(&h->bar_count) - target) < 0) {
                 if (globaltimer_ns() - t0 > kWaitLimitNs) {
                     ok = 0;
                     record_timeout(&h->status);
@@ -380,19 +379,24 @@ __device__ bool grid_barrier(WsHeader *h, uint32_t gen) {
     return s_ok != 0;
 }
 
-template <int T, int V>
+// kOneRound: every row has its own team (M <= teams in the grid), which
+// keeps its row in registers from phase A to phase B.
+template <int T, int V, bool kOneRound>
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(QuantizeArgs a, int64_t kwords) {
     extern __shared__ uint32_t smem[];
     __shared__ uint32_t red[kWarps];
-    __shared__ uint32_t s_gen;
+    __shared__ uint32_t s_gen, s_base;
     uint32_t *bits = smem;                                         // [kwords]
     int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
     const int teams_total = gridDim.x * (kThreads / T);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     // This launch's bitmap is bitmaps[gen & 1]; the previous launch zeroed it.
-    if (threadIdx.x == 0) s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
+    if (threadIdx.x == 0) {
+        s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
+        s_base = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qbase);
+    }
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) bits[w] = 0;
     __syncthreads();
     const uint32_t gen = s_gen;
@@ -401,30 +405,21 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
         nxt[i] = 0;
 
-    // With one row (or none) per team, the team keeps its row in registers
-    // from phase A to phase B instead of reading it twice.
     constexpr int kTeams = kThreads / T;
     const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
-    const bool one_round = V > 0 && a.M <= teams_total;
     const int64_t my_row = (int64_t)blockIdx.x * kTeams + team;
-    uint4 xr[V > 0 ? V : 1];
+    uint4 xr[kOneRound ? V : 1];
 
     // Phase A: O = { h : some |X[i,h]| >= threshold } over every row.
-    if (one_round) {
-        if constexpr (V > 0) {
-            const int64_t nvec = a.K / 8;
+    if constexpr (kOneRound) {
+        if (my_row < a.M) {
+            const int nvec = (int)(a.K / 8);
             const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
-            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + my_row * a.K);
+            load_row<T, V>(a, my_row, tl, xr);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                xr[i] = (my_row < a.M && v < nvec) ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int64_t v = tl + (int64_t)i * T;
-                const uint32_t b = (my_row < a.M && v < nvec) ? outlier_byte(xr[i], t2) : 0u;
-                if (b) atomicOr(&bits[(v * 8) >> 5], b << ((v * 8) & 31));
+                const int v = tl + i * T;
+                if (v < nvec) flag_vec(xr[i], t2, v, bits);
             }
         }
     } else {
@@ -433,7 +428,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
     __syncthreads();
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
         if (bits[w]) atomicOr(&cur[w], bits[w]);
-    if (!grid_barrier(a.hdr, gen)) return;  // every CTA waits in the same barrier
+    if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
 
     // Phase B: codes, scales, outlier activations; outlier-weight gather.
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
@@ -457,26 +452,40 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
             }
         }
     }
-    if (one_round) {
-        if constexpr (V > 0) quantize_row_regs<T, V>(a, bits, prefix, n_out, xr, my_row, my_row < a.M, red, team, tl);
-    } else {
+    if constexpr (kOneRound)
+        quantize_row_regs<T, V>(a, bits, prefix, n_out, xr, my_row, my_row < a.M, red, team, tl);
+    else
         quantize_rows_team<T, V>(a, bits, prefix, n_out, gridDim.x, red);
-    }
     if (a.Wo) {
-        for (int64_t j = (int64_t)blockIdx.x * kWarps + warp; j < a.N; j += (int64_t)gridDim.x * kWarps) {
-            __half *wo = a.Wo + j * a.kcap;
-            for (int32_t t = lane; t < n16; t += 32) {
-                __half val = __float2half_rn(0.f);
-                if (t < n_out) {
-                    const int64_t col = outlier_column(bits, prefix, kwords, t);
-                    if (a.W_outlier) {
-                        val = a.W_outlier[j * a.K + col];
-                    } else {
-                        const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
-                        val = __float2half_rn(__fdiv_rn(p, 127.f));
+        // Wo[j, t] = W[j, col_t]: half-warps over output channels, a lane per
+        // outlier rank t, four channels' loads in flight before any store.
+        const int hl = lane & 15;
+        const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
+        const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
+        for (int32_t t0 = 0; t0 < n16; t0 += 16) {
+            const int32_t t = t0 + hl;
+            const bool real = t < n_out;
+            const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
+            for (int64_t j0 = hw; j0 < a.N; j0 += 4 * nhw) {
+                __half val[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t j = j0 + u * nhw;
+                    val[u] = __float2half_rn(0.f);
+                    if (real && j < a.N) {
+                        if (a.W_outlier) {
+                            val[u] = a.W_outlier[j * a.K + col];
+                        } else {
+                            const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
+                            val[u] = __float2half_rn(__fdiv_rn(p, 127.f));
+                        }
                     }
                 }
-                wo[t] = val;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t j = j0 + u * nhw;
+                    if (j < a.N) a.Wo[j * a.kcap + t] = val[u];
+                }
             }
         }
     }
@@ -516,7 +525,7 @@ namespace {
 
 // Resident CTAs of one kernel instance on the current device (for the
 // cooperative grid size), computed once per device.
-template <int T, int V>
+template <int T, int V, bool R>
 cudaError_t resident_ctas(size_t smem, int *out) {
     static std::once_flag once[64];
     static int count[64];
@@ -527,10 +536,10 @@ cudaError_t resident_ctas(size_t smem, int *out) {
     dev &= 63;
     std::call_once(once[dev], [&] {
         int per_sm = 0, sms = 0;
-        err[dev] = cudaFuncSetAttribute(quantize_kernel<T, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err[dev] = cudaFuncSetAttribute(quantize_kernel<T, V, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)(2 * kMaxKwords * 4));
         if (err[dev] == cudaSuccess)
-            err[dev] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel<T, V>, kThreads,
+            err[dev] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel<T, V, R>, kThreads,
                                                                      2 * kMaxKwords * 4);
         if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         count[dev] = per_sm * sms;
@@ -540,11 +549,26 @@ cudaError_t resident_ctas(size_t smem, int *out) {
     return err[dev];
 }
 
+template <int T, int V, bool R>
+cudaError_t launch_quantize_tvr(const QuantizeArgs &a, int64_t kwords, int grid, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)kwords * 8;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_kernel<T, V, R>, a, kwords);
+}
+
 template <int T, int V>
 cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, cudaStream_t s) {
     const size_t smem = (size_t)kwords * 8;
     int max_ctas = 0;
-    if (cudaError_t e = resident_ctas<T, V>(smem, &max_ctas)) return e;
+    if (cudaError_t e = resident_ctas<T, V, false>(smem, &max_ctas)) return e;
     if (max_ctas <= 0) return cudaErrorInvalidConfiguration;
     const int teams = kThreads / T;
     // Enough teams for every row where possible; the grid barrier needs every
@@ -552,17 +576,16 @@ cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, cudaStream
     int64_t want = ceil_div(a.M, teams);
     if (a.Wo) want = std::max<int64_t>(want, std::min<int64_t>(ceil_div(a.N, kWarps), 148));
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quantize_kernel<T, V>, a, kwords);
+    if constexpr (V > 0) {
+        // One round (each row its own team) needs a grid that covers every row.
+        int max_r = 0;
+        if (cudaError_t e = resident_ctas<T, V, true>(smem, &max_r)) return e;
+        const int64_t need = ceil_div(a.M, teams);
+        if (need <= max_r)
+            return launch_quantize_tvr<T, V, true>(a, kwords, (int)std::max<int64_t>(need, grid > max_r ? max_r : grid),
+                                                   s);
+    }
+    return launch_quantize_tvr<T, V, false>(a, kwords, grid, s);
 }
 
 }  // namespace

@@ -204,6 +204,19 @@ int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t
                           int32_t *C, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Test entry (host only, no GPU needed): the work schedule of the prefill
+ * GEMM for `tiles` output tiles of `nkb` 128-byte k-blocks over `pairs` CTA
+ * pairs, as the kernel walks it. Writes up to cap_rows rows of 6 int32
+ * (pair, tile, first k-block, end k-block, head flag, tail flag) and returns
+ * the number of segments (or -1 for bad arguments). Whole tiles go round-
+ * robin; when the tile count is not a multiple of the pair count, the last
+ * tiles are split into equal k-block ranges, one per pair, and a split
+ * tile's head (its first k-blocks, which finishes it) and tail (its last
+ * k-blocks, whose int32 sums are handed over) sit in adjacent pairs.
+ */
+int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int32_t *out, int cap_rows);
+
+/*
  * Test entry: launch one block that waits on a barrier nothing ever arrives
  * at, with the same bounded-wait routine the GEMM pipeline uses, limited to
  * `limit_ns` nanoseconds (1e3 .. 1e9). The kernel records INT8LT_ERR_TIMEOUT

@@ -1,0 +1,73 @@
+"""The prefill GEMM's tile schedule (data-parallel + stream-K), on the CPU.
+
+int8lt_debug_gemm_schedule enumerates, on the host, the exact segments the
+kernel walks. Every (tile, k-block) must be computed exactly once; a split
+tile has one head (from k-block 0, finishing the tile) in pair p and one
+tail (to the last k-block, handing its int32 sums over) in pair p + 1; the
+k-blocks per pair differ by at most one tile's worth in the data-parallel
+part and by at most one k-block in the stream-K part.
+"""
+import numpy as np
+import pytest
+
+from bit_quantized_matmul_int8_b200 import _lib, build
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def schedule(L, tiles, nkb, pairs):
+    n = L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, None, 0)
+    out = np.zeros((max(n, 1), 6), np.int32)
+    assert L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, out.ctypes.data, n) == n
+    return out[:n]
+
+
+@pytest.mark.parametrize("tiles,nkb,pairs", [
+    (128, 32, 74),      # 2048 x 4096 x 4096 on 74 pairs: 1.73 waves
+    (1024, 32, 74),     # 4096 x 4096 x 16384
+    (256, 128, 74),     # 4096 x 16384 x 4096
+    (1152, 96, 74),     # 8192 x 12288 x 36864
+    (74, 32, 74), (148, 8, 74), (3, 5, 3), (1, 1, 1), (7, 1, 4), (10, 3, 4), (75, 2, 74),
+])
+def test_schedule_covers_every_kblock_once(L, tiles, nkb, pairs):
+    s = schedule(L, tiles, nkb, pairs)
+    cover = np.zeros((tiles, nkb), np.int32)
+    for p, t, k0, k1, head, tail in s:
+        assert 0 <= t < tiles and 0 <= k0 < k1 <= nkb
+        cover[t, k0:k1] += 1
+        assert head == (k0 == 0 and k1 < nkb)
+        assert tail == (k0 > 0)
+        if tail:
+            assert k1 == nkb
+    assert (cover == 1).all()
+    heads = {t: p for p, t, k0, k1, h, tl in s if h}
+    tails = {t: p for p, t, k0, k1, h, tl in s if tl}
+    assert heads.keys() == tails.keys()
+    for t in heads:
+        assert tails[t] == heads[t] + 1
+    # a pair owns at most one head, as its last segment, and at most one tail,
+    # as the first segment of its stream-K range (after its whole tiles, whose
+    # count is the same for every pair, so the tail is ready long before the
+    # head of the previous pair needs it)
+    for p in range(pairs):
+        mine = s[s[:, 0] == p]
+        if len(mine):
+            assert mine[:-1, 4].sum() == 0 and mine[:, 5].sum() <= 1
+            if mine[:, 5].any():
+                k = int(np.nonzero(mine[:, 5])[0][0])
+                assert (mine[k + 1:, 1] > mine[k, 1]).all()
+                assert (mine[:k, 2] == 0).all() and (mine[:k, 3] == nkb).all()
+    # balance: stream-K k-blocks per pair differ by at most one
+    work = np.array([(s[s[:, 0] == p, 3] - s[s[:, 0] == p, 2]).sum() for p in range(pairs)])
+    if tiles % pairs and tiles > pairs:
+        assert work.max() - work.min() <= 1
+    assert work.sum() == tiles * nkb
+
+
+def test_bad_arguments(L):
+    assert L.int8lt_debug_gemm_schedule(4, 0, 2, None, 0) == -1
+    assert L.int8lt_debug_gemm_schedule(4, 2, 0, None, 0) == -1

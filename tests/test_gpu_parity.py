@@ -107,6 +107,20 @@ def test_gemm_int32_bit_exact(M, N, K):
     assert np.array_equal(C.astype(np.int64), ref)
 
 
+# Tile counts above the resident CTA-pair count and not a multiple of it: the
+# last tiles are split between two pairs (head + tail with int32 partials).
+SPLIT_SHAPES = [(1280, 4096, 512), (2048, 4096, 384), (2304, 4352, 1152)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+def test_gemm_int32_split_tiles_bit_exact(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    assert np.array_equal(C, oracle.gemm_i32(A, B))
+
+
 def test_gemm_int32_matches_oracle_routine():
     rng = np.random.default_rng(9)
     A = rng.integers(-127, 128, (200, 336), dtype=np.int64).astype(np.int8)
@@ -144,6 +158,20 @@ def test_forward_vs_oracle(w, thr):
     t = w.threshold if thr == "cfg" else math.inf
     X, W, b = case_inputs(w)
     Yg, Y64 = run_forward(X, W, b, t)
+    check_y(Yg, Y64, w.name)
+
+
+SPLIT_FCASES = [
+    wl.random_case(59, 1280, 512, 4096, n_outliers=6, frac=0.5),
+    wl.random_case(60, 2048, 384, 4096, n_outliers=45, frac=0.3),   # two outlier k-blocks
+    wl.random_case(61, 1280, 640, 4096, n_outliers=0, has_bias=False),
+]
+
+
+@pytest.mark.parametrize("w", SPLIT_FCASES, ids=[w.name for w in SPLIT_FCASES])
+def test_forward_split_tiles_vs_oracle(w):
+    X, W, b = case_inputs(w)
+    Yg, Y64 = run_forward(X, W, b, w.threshold)
     check_y(Yg, Y64, w.name)
 
 
