@@ -27,7 +27,7 @@ EXPORTS = [
     "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
-    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout",
+    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
 ]
 
 
@@ -56,7 +56,8 @@ _SIGS = {
     "int8lt_forward_static_scratch": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P]),
     "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
-    "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
+    "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
+    "int8lt_set_gemm_split": (ctypes.c_int, [ctypes.c_int]),
 }
 
 
@@ -250,6 +251,17 @@ def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, ws: torch.Tensor |
 def int8lt_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
     _check("int8lt_debug_wait_timeout",
            lib().int8lt_debug_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
+
+
+SPLIT_AUTO, SPLIT_ALWAYS, SPLIT_NEVER = 0, 1, 2
+
+
+def int8lt_set_gemm_split(mode: int) -> int:
+    """Set the prefill GEMM's split policy (SPLIT_*); returns the previous one."""
+    prev = int(lib().int8lt_set_gemm_split(int(mode)))
+    if prev < 0:
+        raise ValueError(f"unknown split mode {mode}")
+    return prev
 
 
 class Int8Linear:

@@ -31,6 +31,7 @@
 // Every wait is bounded (kWaitLimitNs); a wait that runs out sets the
 // workspace status word and the kernel winds down without touching Y.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "int8lt_internal.cuh"
@@ -88,6 +89,20 @@ struct TileSched {
         return true;
     }
 };
+
+// Split policy (INT8LT_SPLIT_*): process-wide, read at each launch.
+std::atomic<int> g_split_mode{0};
+
+// Whether the tiles after the last full wave are split between pairs. Auto:
+// only when it saves the busiest pair at least 32 k-blocks, roughly the
+// measured cost of handing the tails' int32 sums over.
+bool split_wanted(int64_t tiles, int nkb, int pairs, int mode) {
+    if (pairs > kSkMaxPairs || tiles <= pairs || tiles % pairs == 0 || mode == 2) return false;
+    if (mode == 1) return true;
+    const int64_t waves = (tiles + pairs - 1) / pairs;
+    const int64_t saved = (waves * pairs - tiles) * (int64_t)nkb / pairs;  // k-blocks per pair
+    return saved >= 32;
+}
 
 namespace {
 
@@ -271,9 +286,6 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const uint32_t rank = cluster_ctarank();          // 0: leader, 1: follower
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const int nkb = (int)ceil_div(a.K, 128);
-    const int n_out = (a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
-    const int n_okb = (n_out + kOkb - 1) / kOkb;       // outlier k-blocks per tile
-    const int n_mma_o = (n_out + 15) >> 4;             // fp16 MMAs of K = 16 per tile
     const bool sk_on = a.sk_partial && a.sk_flags && num_pairs <= kSkMaxPairs;
 
     if (threadIdx.x == 0) {
@@ -299,10 +311,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tma_prefetch(&tmA);
         tma_prefetch(&tmB);
         if (!a.C32) tma_prefetch(&tmY);
-        if (n_okb) {
-            tma_prefetch(&tmXo);
-            tma_prefetch(&tmWo);
-        }
+        tma_prefetch(&tmXo);
+        tma_prefetch(&tmWo);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(&ctrl->tmem_base), kTmemCols);
@@ -312,6 +322,13 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncthreads();
     cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
     tc_fence_after();
+    // Everything above touches only this CTA pair; from here on the kernel
+    // reads what the quantize pass wrote (launched with programmatic stream
+    // serialization, the prologue overlaps the end of that pass).
+    grid_dep_wait();
+    const int n_out = (a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
+    const int n_okb = (n_out + kOkb - 1) / kOkb;       // outlier k-blocks per tile
+    const int n_mma_o = (n_out + 15) >> 4;             // fp16 MMAs of K = 16 per tile
     const uint32_t tmem = ctrl->tmem_base;
     volatile uint32_t *abort_flag = &ctrl->abort;
 
@@ -737,11 +754,13 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     cudaError_t attr_err = cudaSuccess;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;  // CTA pairs
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = s;
@@ -761,19 +780,27 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     const int num_m_tiles = (int)ceil_div(a.M, BM);
     const int64_t tiles = (int64_t)num_m_tiles * ceil_div(a.N, BN);
     const int pairs = g_num_sms[dev & 63] > 0 ? g_num_sms[dev & 63] : 74;
-    cfg.gridDim = dim3(2 * (unsigned)std::min<int64_t>(tiles, pairs), 1, 1);
-    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, mY, a, num_m_tiles, (int)tiles);
+    const int grid_pairs = (int)std::min<int64_t>(tiles, pairs);
+    GemmArgs b = a;
+    if (!split_wanted(tiles, (int)ceil_div(a.K, 128), grid_pairs, g_split_mode.load(std::memory_order_relaxed))) {
+        b.sk_partial = nullptr;
+        b.sk_flags = nullptr;
+    }
+    cfg.gridDim = dim3(2 * (unsigned)grid_pairs, 1, 1);
+    cfg.numAttrs = 2;  // and programmatic stream serialization
+    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, mY, b, num_m_tiles, (int)tiles);
 }
 
 }  // namespace int8lt
 
-// Test entry: the stream-K schedule as the GEMM walks it, enumerated on the
-// host. Rows of 6 int32: pair, tile, kb0, kb1, head, tail.
-extern "C" int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int32_t *out, int cap_rows) {
-    if (tiles < 0 || nkb < 1 || pairs < 1 || (!out && cap_rows > 0)) return -1;
+// Test entry: the schedule as the GEMM walks it, enumerated on the host.
+// Rows of 6 int32: pair, tile, kb0, kb1, head, tail.
+extern "C" int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int mode, int32_t *out, int cap_rows) {
+    if (tiles < 0 || nkb < 1 || pairs < 1 || mode < 0 || mode > 2 || (!out && cap_rows > 0)) return -1;
+    const bool sk = int8lt::split_wanted(tiles, nkb, pairs, mode);
     int n = 0;
     for (int p = 0; p < pairs; ++p) {
-        int8lt::TileSched ts(tiles, nkb, nkb, pairs, p, pairs <= int8lt::kSkMaxPairs);
+        int8lt::TileSched ts(tiles, nkb, nkb, pairs, p, sk);
         int8lt::Seg g;
         while (ts.next(g)) {
             if (n < cap_rows) {
@@ -784,4 +811,9 @@ extern "C" int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int32_t
         }
     }
     return n;
+}
+
+extern "C" int int8lt_set_gemm_split(int mode) {
+    if (mode < 0 || mode > 2) return -1;
+    return int8lt::g_split_mode.exchange(mode);
 }

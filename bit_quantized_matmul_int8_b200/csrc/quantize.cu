@@ -5,20 +5,21 @@
 // Core of LLM.int8(): Mixed-precision Decomposition"; "Hugging Face LLM.int8()
 // integration" (agentlenshq.com), three-step recipe and CB/SCB weights.
 //
-// Kernels (all HBM-bound streaming passes with 16-byte coalesced loads):
+// Kernels (HBM-bound streaming passes):
 //   prepare_weight_kernel  W [N,K] -> CB, SCB          (one warp per row)
-//   quantize_kernel        one cooperative launch: phase A ORs the outlier
-//                          columns of every row into a bitmap, a grid
-//                          barrier, then phase B writes O, CA, SCA, Xo,
-//                          gathers Wo and clears the split-K buffers of the
-//                          GEMV
+//   quantize_kernel        one cooperative launch: the CTA's rows of X are
+//                          staged in shared memory by bulk copies; phase A
+//                          ORs the outlier columns of every row into a
+//                          bitmap, a grid barrier, then phase B writes O, CA,
+//                          SCA, Xo from the staged rows, gathers Wo and
+//                          clears the split-K buffers of the GEMV
 //
 // Exactness: |x| >= threshold is decided on the fp16 bit pattern against the
 // smallest fp16 pattern whose value reaches the fp32 threshold (the map from
 // non-negative fp16 patterns to values is monotonic, so this is the fp32
 // comparison). The absmax is a max of fp16 magnitudes (exact). The code is
-// rint(x * fp32(127 / absmax)) with __fdiv_rn / __fmul_rn / __float2int_rn:
-// one IEEE rounding per step, ties to even, never contracted into an FMA.
+// rint(x * fp32(127 / absmax)) with __fdiv_rn / __fmul_rn and a rounding
+// add: one IEEE rounding per step, ties to even, never contracted into an FMA.
 #include <algorithm>
 #include <mutex>
 
@@ -30,6 +31,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 16;  // 16-byte loads in flight per thread in phase A
 
 // Code of x: rint(fp32(x * s)) with s = fp32(127 / absmax) and |x| <= absmax.
 // No clamp is needed: |x * s| <= 127 * (1 + 2^-23) before rounding, so the
@@ -164,8 +166,6 @@ __device__ __forceinline__ uint32_t vec_mask(const uint32_t *bits, int v) {
     return (bits[v >> 2] >> ((v & 3) * 8)) & 0xffu;
 }
 
-// Slow paths for the few vectors holding outlier columns, kept out of line
-// so the unrolled fast path does not reserve registers for them.
 // Phase A test of one vector of 8 halves: set bit (v*8 + k) of `bits` for
 // every element k with |x| >= threshold (t2 = the threshold's binary16 bits,
 // twice). A vector with no hit, the usual case, costs four compares.
@@ -178,164 +178,90 @@ __device__ __forceinline__ void flag_vec(uint4 x, uint32_t t2, int v, uint32_t *
     atomicOr(&bits[v >> 2], b << ((v & 3) * 8));
 }
 
-__device__ __noinline__ uint32_t masked_absmax_bits_slow(uint4 x, uint32_t m) {
-    const uint16_t *e = reinterpret_cast<const uint16_t *>(&x);
-    uint32_t amax = 0;
+// The vector with its outlier elements (bits of m) replaced by +0: their
+// code is then 0 and they do not count in the absmax.
+__device__ __forceinline__ uint4 clear_masked(uint4 x, uint32_t m) {
+    uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        if (!((m >> j) & 1u)) amax = max(amax, (uint32_t)(e[j] & 0x7fffu));
-    return amax;
-}
-
-__device__ __forceinline__ uint32_t masked_absmax_bits(uint4 x, uint32_t m) {
-    return m == 0 ? vec_absmax_bits(x) : masked_absmax_bits_slow(x, m);
-}
-
-// Codes of vector v (outlier columns -> 0, and their fp16 values -> Xo).
-__device__ __noinline__ uint2 quant_masked_slow(uint4 x, uint32_t m, float s, int v, const uint32_t *bits,
-                                                const int32_t *prefix, __half *xo) {
-    uint2 q = quant_vec8(x, s);
-    {
-        const __half *e = reinterpret_cast<const __half *>(&x);
-        uint32_t keep0 = 0, keep1 = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if ((m >> j) & 1u) {
-                if (xo) {
-                    const int col = v * 8 + j;
-                    const int32_t rank = prefix[col >> 5] + __popc(bits[col >> 5] & ((1u << (col & 31)) - 1u));
-                    xo[rank] = e[j];
-                }
-            } else {
-                if (j < 4) keep0 |= 0xffu << (8 * j); else keep1 |= 0xffu << (8 * (j - 4));
-            }
-        }
-        q.x &= keep0;
-        q.y &= keep1;
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = ((m >> (2 * j)) & 1u) ? 0u : 0x0000ffffu;
+        const uint32_t hi = ((m >> (2 * j + 1)) & 1u) ? 0u : 0xffff0000u;
+        w[j] &= lo | hi;
     }
-    return q;
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ uint2 quant_masked(uint4 x, uint32_t m, float s, int v, const uint32_t *bits,
-                                              const int32_t *prefix, __half *xo) {
-    return m == 0 ? quant_vec8(x, s) : quant_masked_slow(x, m, s, v, bits, prefix, xo);
+// Xo[rank of column] = x for the outlier elements (bits of m) of vector v.
+__device__ __forceinline__ void store_outliers(uint4 x, uint32_t m, int v, const uint32_t *bits,
+                                               const int32_t *prefix, __half *xo) {
+    while (m) {
+        const int j = __ffs(m) - 1;
+        m &= m - 1;
+        const uint32_t w = j < 4 ? (j < 2 ? x.x : x.y) : (j < 6 ? x.z : x.w);
+        const unsigned short h = (unsigned short)((j & 1) ? (w >> 16) : (w & 0xffffu));
+        const int col = v * 8 + j;
+        xo[prefix[col >> 5] + __popc(bits[col >> 5] & ((1u << (col & 31)) - 1u))] = __ushort_as_half(h);
+    }
 }
 
-// Max over the T threads of a row team (T = 32: one warp; T = 128: four
-// warps synchronised by a named barrier private to the team).
-template <int T>
-__device__ __forceinline__ uint32_t team_max(uint32_t v, uint32_t *red, int team) {
-    v = warp_max_u32(v);
-    if (T == 32) return v;
-    const int tw = (threadIdx.x & (T - 1)) >> 5;
-    if ((threadIdx.x & 31) == 0) red[team * (T / 32) + tw] = v;
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(T) : "memory");
-    uint32_t r = red[team * (T / 32)];
-#pragma unroll
-    for (int i = 1; i < T / 32; ++i) r = max(r, red[team * (T / 32) + i]);
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(T) : "memory");  // red reusable
-    return r;
+// One warp per row. `row` points at the row's nvec 16-byte vectors, in
+// shared memory (kSmem) or in X. Loops are rolled (unroll 4): the kernel's
+// code stays small enough for the instruction caches.
+template <bool kSmem>
+__device__ __forceinline__ uint4 ld_vec(const uint4 *p) {
+    if constexpr (kSmem) return *p;
+    else return __ldg(p);
 }
 
-// One row per team of T threads; the team's row is held in V 16-byte
-// registers per thread (V * T * 8 >= K), or re-read when V == 0.
-// Phase B of one row held in registers (V > 0): masked absmax over the team,
-// codes, scale and outlier activations. Every thread of the team calls it.
-template <int T, int V>
-__device__ __forceinline__ void quantize_row_regs(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
-                                                  int32_t n_out, const uint4 (&x)[V], int64_t r, bool valid,
-                                                  uint32_t *red, int team, int tl) {
+// Phase B of row r: masked absmax, codes, scale and outlier activations.
+// Vectors holding outlier columns (a handful per row) take a short branch.
+template <bool kSmem>
+__device__ __forceinline__ void quantize_row(const QuantizeArgs &a, const uint4 *row, int64_t r, const uint32_t *bits,
+                                             const int32_t *prefix, int32_t n_out, int lane) {
     const int nvec = (int)(a.K / 8);
-    const int32_t n16 = (n_out + 15) & ~15;
-    uint32_t m[V];
     uint32_t amax = 0;
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int v = tl + i * T;
-        const bool in = valid && v < nvec;
-        m[i] = in ? vec_mask(bits, v) : 0u;
-        if (in) amax = max(amax, masked_absmax_bits(x[i], m[i]));
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) {
+        uint4 x = ld_vec<kSmem>(row + v);
+        const uint32_t m = vec_mask(bits, v);
+        if (m) x = clear_masked(x, m);
+        amax = max(amax, vec_absmax_bits(x));
     }
-    amax = team_max<T>(amax, red, team);
-    if (!valid) return;
+    amax = warp_max_u32(amax);
     const float sa = __half2float(__ushort_as_half((unsigned short)amax));
     const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
     uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
     __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int v = tl + i * T;
-        if (v < nvec) ca2[v] = quant_masked(x[i], m[i], s, v, bits, prefix, xo);
-    }
-    if (xo)
-        for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
-    if (tl == 0) a.SCA[r] = sa;
-}
-
-// Load the V vectors of row r a team thread owns (zeros past the row end).
-template <int T, int V>
-__device__ __forceinline__ void load_row(const QuantizeArgs &a, int64_t r, int tl, uint4 (&x)[V]) {
-    const int nvec = (int)(a.K / 8);
-    const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int v = tl + i * T;
-        x[i] = v < nvec ? __ldg(x4 + v) : make_uint4(0, 0, 0, 0);
-    }
-}
-
-// Phase B for the team's rows, re-read from memory (rows are not kept).
-template <int T, int V>
-__device__ void quantize_rows_team(const QuantizeArgs &a, const uint32_t *bits, const int32_t *prefix,
-                                   int32_t n_out, int row_ctas, uint32_t *red) {
-    const int teams = kThreads / T;
-    const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
-    for (int64_t r = (int64_t)blockIdx.x * teams + team; r < a.M; r += (int64_t)row_ctas * teams) {
-        if constexpr (V > 0) {
-            uint4 x[V];
-            load_row<T, V>(a, r, tl, x);
-            quantize_row_regs<T, V>(a, bits, prefix, n_out, x, r, true, red, team, tl);
-        } else {
-            const int nvec = (int)(a.K / 8);
-            const int32_t n16 = (n_out + 15) & ~15;
-            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
-            uint32_t amax = 0;
-            for (int v = tl; v < nvec; v += T) amax = max(amax, masked_absmax_bits(__ldg(x4 + v), vec_mask(bits, v)));
-            amax = team_max<T>(amax, red, team);
-            const float sa = __half2float(__ushort_as_half((unsigned short)amax));
-            const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
-            uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
-            __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
-            for (int v = tl; v < nvec; v += T)
-                ca2[v] = quant_masked(__ldg(x4 + v), vec_mask(bits, v), s, v, bits, prefix, xo);
-            if (xo)
-                for (int32_t t = n_out + tl; t < n16; t += T) xo[t] = __float2half_rn(0.f);
-            if (tl == 0) a.SCA[r] = sa;
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) {
+        uint4 x = ld_vec<kSmem>(row + v);
+        const uint32_t m = vec_mask(bits, v);
+        if (m) {
+            if (xo) store_outliers(x, m, v, bits, prefix, xo);
+            x = clear_masked(x, m);
         }
+        ca2[v] = quant_vec8(x, s);
     }
+    if (xo) {
+        const int32_t n16 = (n_out + 15) & ~15;
+        for (int32_t t = n_out + lane; t < n16; t += 32) xo[t] = __float2half_rn(0.f);
+    }
+    if (lane == 0) a.SCA[r] = sa;
 }
 
-// Phase A for one team's rows: OR the rows' outlier bits into the CTA bitmap.
-template <int T, int V>
-__device__ void flag_rows_team(const QuantizeArgs &a, uint32_t *bits, int teams_total) {
-    const int teams = kThreads / T;
-    const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
+// Phase B of a staged row whose outlier elements are already zero.
+__device__ __forceinline__ void quantize_row_plain(const QuantizeArgs &a, const uint4 *row, int64_t r, int lane) {
     const int nvec = (int)(a.K / 8);
-    const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
-    for (int64_t r = (int64_t)blockIdx.x * teams + team; r < a.M; r += teams_total) {
-        if constexpr (V > 0) {
-            uint4 x[V];
-            load_row<T, V>(a, r, tl, x);
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int v = tl + i * T;
-                if (v < nvec) flag_vec(x[i], t2, v, bits);
-            }
-        } else {
-            const uint4 *x4 = reinterpret_cast<const uint4 *>(a.X + r * a.K);
-            for (int v = tl; v < nvec; v += T) flag_vec(__ldg(x4 + v), t2, v, bits);
-        }
-    }
+    uint32_t amax = 0;
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) amax = max(amax, vec_absmax_bits(row[v]));
+    amax = warp_max_u32(amax);
+    const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+    const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+    uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) ca2[v] = quant_vec8(row[v], s);
+    if (lane == 0) a.SCA[r] = sa;
 }
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
@@ -379,18 +305,27 @@ __device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base) {
     return s_ok != 0;
 }
 
-// kOneRound: every row has its own team (M <= teams in the grid), which
-// keeps its row in registers from phase A to phase B.
-template <int T, int V, bool kOneRound>
+// Phase A walks the CTA's rows in rounds of R rows (rows of a round are
+// contiguous in X): every thread keeps 16 16-byte loads in flight, tests
+// them and, in the last round, also keeps them in shared memory. Phase B
+// quantizes the last round from shared memory and the earlier rounds from X
+// again (from L2 when X fits); with a single round X is read from HBM
+// exactly once. R = 0 (rows too long to keep): phase B reads every row from X.
 __global__ void __launch_bounds__(kThreads, 2)
-quantize_kernel(QuantizeArgs a, int64_t kwords) {
-    extern __shared__ uint32_t smem[];
-    __shared__ uint32_t red[kWarps];
+quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
+    extern __shared__ __align__(128) uint32_t smem[];
     __shared__ uint32_t s_gen, s_base;
     uint32_t *bits = smem;                                         // [kwords]
     int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
-    const int teams_total = gridDim.x * (kThreads / T);
+    uint4 *rows = reinterpret_cast<uint4 *>(smem + ((2 * kwords + 31) & ~int64_t(31)));  // [R][nvec]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = (int)(a.K / 8);
+    const int rows_per_round = R > 0 ? R : kWarps;
+    const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
+    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
+    // The GEMM behind this pass may start its prologue on SMs this grid frees;
+    // it waits for the whole pass before it reads anything.
+    grid_dep_launch();
 
     // This launch's bitmap is bitmaps[gen & 1]; the previous launch zeroed it.
     if (threadIdx.x == 0) {
@@ -405,25 +340,35 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
         nxt[i] = 0;
 
-    constexpr int kTeams = kThreads / T;
-    const int team = threadIdx.x / T, tl = threadIdx.x & (T - 1);
-    const int64_t my_row = (int64_t)blockIdx.x * kTeams + team;
-    uint4 xr[kOneRound ? V : 1];
-
     // Phase A: O = { h : some |X[i,h]| >= threshold } over every row.
-    if constexpr (kOneRound) {
-        if (my_row < a.M) {
-            const int nvec = (int)(a.K / 8);
-            const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
-            load_row<T, V>(a, my_row, tl, xr);
+    for (int rd = 0; rd < rounds; ++rd) {
+        const int64_t r0 = ((int64_t)rd * gridDim.x + blockIdx.x) * rows_per_round;
+        const int64_t left = a.M - r0;
+        const int nr = left <= 0 ? 0 : (left < rows_per_round ? (int)left : rows_per_round);
+        const bool keep = R > 0 && rd == rounds - 1;
+        const int64_t total = (int64_t)nr * nvec;          // this round's vectors
+        const uint4 *src = X4 + r0 * nvec;
+        int v = threadIdx.x % nvec;                          // column vector of `flat`
+        for (int64_t flat = threadIdx.x; flat < total; flat += kBatch * kThreads) {
+            uint4 x[kBatch];
+            int vs[kBatch];
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                const int v = tl + i * T;
-                if (v < nvec) flag_vec(xr[i], t2, v, bits);
+            for (int u = 0; u < kBatch; ++u) {
+                const int64_t f = flat + u * kThreads;
+                vs[u] = v;
+                x[u] = f < total ? __ldg(src + f) : make_uint4(0, 0, 0, 0);
+                v += kThreads;
+                if (v >= nvec) v = nvec >= kThreads ? v - nvec : v % nvec;
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int64_t f = flat + u * kThreads;
+                if (f < total) {
+                    flag_vec(x[u], t2, vs[u], bits);
+                    if (keep) rows[f] = x[u];
+                }
             }
         }
-    } else {
-        flag_rows_team<T, V>(a, bits, teams_total);
     }
     __syncthreads();
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
@@ -452,10 +397,33 @@ quantize_kernel(QuantizeArgs a, int64_t kwords) {
             }
         }
     }
-    if constexpr (kOneRound)
-        quantize_row_regs<T, V>(a, bits, prefix, n_out, xr, my_row, my_row < a.M, red, team, tl);
-    else
-        quantize_rows_team<T, V>(a, bits, prefix, n_out, gridDim.x, red);
+    for (int rd = rounds - 1; rd >= 0; --rd) {
+        const int64_t r0 = ((int64_t)rd * gridDim.x + blockIdx.x) * rows_per_round;
+        const int64_t left = a.M - r0;
+        const int nr = left <= 0 ? 0 : (left < rows_per_round ? (int)left : rows_per_round);
+        for (int r = warp; r < nr; r += kWarps) {
+            if (R > 0 && rd == rounds - 1) {
+                // Staged row: copy its outlier elements to Xo and zero them
+                // in place, then quantize it without masks.
+                uint4 *row = rows + (size_t)r * nvec;
+                __half *rh = reinterpret_cast<__half *>(row);
+                __half *xo = a.Xo ? a.Xo + (r0 + r) * a.kcap : nullptr;
+                for (int32_t t = lane; t < n16; t += 32) {
+                    __half val = __float2half_rn(0.f);
+                    if (t < n_out) {
+                        const int64_t col = outlier_column(bits, prefix, kwords, t);
+                        val = rh[col];
+                        rh[col] = __ushort_as_half((unsigned short)0);
+                    }
+                    if (xo) xo[t] = val;
+                }
+                __syncwarp();
+                quantize_row_plain(a, row, r0 + r, lane);
+            } else {
+                quantize_row<false>(a, X4 + (r0 + r) * nvec, r0 + r, bits, prefix, n_out, lane);
+            }
+        }
+    }
     if (a.Wo) {
         // Wo[j, t] = W[j, col_t]: half-warps over output channels, a lane per
         // outlier rank t, four channels' loads in flight before any store.
@@ -523,90 +491,85 @@ cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t 
 
 namespace {
 
-// Resident CTAs of one kernel instance on the current device (for the
-// cooperative grid size), computed once per device.
-template <int T, int V, bool R>
-cudaError_t resident_ctas(size_t smem, int *out) {
-    static std::once_flag once[64];
-    static int count[64];
-    static cudaError_t err[64];
+// Largest dynamic shared memory a CTA may ask for while two still fit on an SM.
+constexpr int kQuantDynMax = 113 * 1024 - 512;
+
+struct QuantOcc {
+    std::mutex mu;
+    bool init = false;
+    cudaError_t err = cudaSuccess;
+    int sms = 0;
+    int cached_dyn[8] = {}, cached_per_sm[8] = {}, n_cached = 0;
+};
+
+// Resident CTAs per SM of quantize_kernel with `dyn` bytes of dynamic shared
+// memory on the current device (cached per device and size).
+cudaError_t quant_resident(int dyn, int *ctas) {
+    static QuantOcc occ[64];
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    dev &= 63;
-    std::call_once(once[dev], [&] {
-        int per_sm = 0, sms = 0;
-        err[dev] = cudaFuncSetAttribute(quantize_kernel<T, V, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)(2 * kMaxKwords * 4));
-        if (err[dev] == cudaSuccess)
-            err[dev] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel<T, V, R>, kThreads,
-                                                                     2 * kMaxKwords * 4);
-        if (err[dev] == cudaSuccess) err[dev] = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        count[dev] = per_sm * sms;
-    });
-    (void)smem;
-    *out = count[dev];
-    return err[dev];
-}
-
-template <int T, int V, bool R>
-cudaError_t launch_quantize_tvr(const QuantizeArgs &a, int64_t kwords, int grid, cudaStream_t s) {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)kwords * 8;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quantize_kernel<T, V, R>, a, kwords);
-}
-
-template <int T, int V>
-cudaError_t launch_quantize_tv(const QuantizeArgs &a, int64_t kwords, cudaStream_t s) {
-    const size_t smem = (size_t)kwords * 8;
-    int max_ctas = 0;
-    if (cudaError_t e = resident_ctas<T, V, false>(smem, &max_ctas)) return e;
-    if (max_ctas <= 0) return cudaErrorInvalidConfiguration;
-    const int teams = kThreads / T;
-    // Enough teams for every row where possible; the grid barrier needs every
-    // CTA resident at once, which the cooperative launch guarantees.
-    int64_t want = ceil_div(a.M, teams);
-    if (a.Wo) want = std::max<int64_t>(want, std::min<int64_t>(ceil_div(a.N, kWarps), 148));
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
-    if constexpr (V > 0) {
-        // One round (each row its own team) needs a grid that covers every row.
-        int max_r = 0;
-        if (cudaError_t e = resident_ctas<T, V, true>(smem, &max_r)) return e;
-        const int64_t need = ceil_div(a.M, teams);
-        if (need <= max_r)
-            return launch_quantize_tvr<T, V, true>(a, kwords, (int)std::max<int64_t>(need, grid > max_r ? max_r : grid),
-                                                   s);
+    if (cudaError_t e = cudaGetDevice(&dev)) return e;
+    QuantOcc &o = occ[dev & 63];
+    std::lock_guard<std::mutex> lock(o.mu);
+    if (!o.init) {
+        o.init = true;
+        o.err = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantDynMax);
+        if (o.err == cudaSuccess) o.err = cudaDeviceGetAttribute(&o.sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    return launch_quantize_tvr<T, V, false>(a, kwords, grid, s);
+    if (o.err != cudaSuccess) return o.err;
+    for (int i = 0; i < o.n_cached; ++i)
+        if (o.cached_dyn[i] == dyn) {
+            *ctas = o.cached_per_sm[i] * o.sms;
+            return cudaSuccess;
+        }
+    int per_sm = 0;
+    if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_kernel, kThreads, dyn)) return e;
+    const int slot = o.n_cached < 8 ? o.n_cached++ : (dyn & 7);
+    o.cached_dyn[slot] = dyn;
+    o.cached_per_sm[slot] = per_sm;
+    *ctas = per_sm * o.sms;
+    return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     const int64_t kwords = ceil_div(a.K, 32);
-    const int64_t nvec = a.K / 8;
-    // Row team: one warp per row up to K = 4096 (up to 16 loads in flight per
-    // lane, and every row of a 2048-token batch in flight at once), four warps
-    // per row up to K = 16384 (the row stays in registers); longer rows are
-    // read twice.
-    const int T = nvec <= 32 * 16 ? 32 : 128;
-    const int64_t v = ceil_div(nvec, T);
-    if (T == 32) {
-        if (v <= 4) return launch_quantize_tv<32, 4>(a, kwords, s);
-        if (v <= 8) return launch_quantize_tv<32, 8>(a, kwords, s);
-        return launch_quantize_tv<32, 16>(a, kwords, s);
+    const int64_t bits_bytes = round_up(2 * kwords * 4, 128);
+    const int64_t row_bytes = 2 * a.K;
+    // Rows kept per CTA and round (0: rows too long to keep; phase B reads X).
+    const int64_t r_max = std::min<int64_t>(64, (kQuantDynMax - bits_bytes) / row_bytes);
+    int R = 0, rounds = 1, grid = 0, resident = 0;
+    if (r_max > 0) {
+        if (cudaError_t e = quant_resident((int)(bits_bytes + r_max * row_bytes), &resident)) return e;
+        if (resident <= 0) return cudaErrorInvalidConfiguration;
+        if (a.M <= r_max * resident) {
+            // One round: spread the rows over every resident CTA.
+            R = (int)ceil_div(a.M, resident);
+            grid = (int)ceil_div(a.M, R);
+        } else {
+            // Several rounds of equal size; the last one stays staged.
+            grid = resident;
+            rounds = (int)ceil_div(a.M, r_max * resident);
+            R = (int)ceil_div(a.M, (int64_t)resident * rounds);
+        }
+    } else {
+        if (cudaError_t e = quant_resident((int)bits_bytes, &resident)) return e;
+        if (resident <= 0) return cudaErrorInvalidConfiguration;
+        grid = (int)std::min<int64_t>(resident, std::max<int64_t>(1, ceil_div(a.M, kWarps)));
+        rounds = (int)ceil_div(a.M, (int64_t)kWarps * grid);  // kWarps rows per CTA and round
     }
-    if (v <= 8) return launch_quantize_tv<128, 8>(a, kwords, s);
-    if (v <= 16) return launch_quantize_tv<128, 16>(a, kwords, s);
-    return launch_quantize_tv<128, 0>(a, kwords, s);
+    // The grid barrier needs every CTA resident at once: a cooperative launch.
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)std::max(grid, 1), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)(bits_bytes + (int64_t)R * row_bytes);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_kernel, a, kwords, R, rounds);
 }
 
 }  // namespace int8lt

@@ -203,18 +203,38 @@ int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N, int64_t K
 int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K,
                           int32_t *C, void *ws, size_t ws_bytes, void *stream);
 
+/* Schedules of the prefill GEMM's last wave (int8lt_set_gemm_split). */
+enum {
+    INT8LT_SPLIT_AUTO = 0,    /* split when it saves enough (default) */
+    INT8LT_SPLIT_ALWAYS = 1,  /* split whenever the tile count allows */
+    INT8LT_SPLIT_NEVER = 2    /* whole tiles only */
+};
+
+/*
+ * Tuning: how the prefill GEMM (M > 16) schedules its 256 x 256 output tiles
+ * over its CTA pairs. Whole tiles go round-robin. When the tile count is not
+ * a multiple of the pair count, the tiles after the last full wave may be
+ * split into equal k-block ranges, one per pair ("stream-K"), at the price of
+ * handing one tile's int32 sums per pair through the workspace (measured at
+ * roughly 8 us per launch). INT8LT_SPLIT_AUTO splits only when that saves the
+ * busiest pair at least 32 k-blocks of 128 bytes (one 256 x 256 x 4096 tile).
+ * The setting is process-wide, thread-safe, and applies to launches made
+ * after the call; the results do not depend on it (integer sums are exact).
+ * Returns the previous mode, or -1 for an unknown mode.
+ */
+int int8lt_set_gemm_split(int mode);
+
 /*
  * Test entry (host only, no GPU needed): the work schedule of the prefill
  * GEMM for `tiles` output tiles of `nkb` 128-byte k-blocks over `pairs` CTA
- * pairs, as the kernel walks it. Writes up to cap_rows rows of 6 int32
- * (pair, tile, first k-block, end k-block, head flag, tail flag) and returns
- * the number of segments (or -1 for bad arguments). Whole tiles go round-
- * robin; when the tile count is not a multiple of the pair count, the last
- * tiles are split into equal k-block ranges, one per pair, and a split
- * tile's head (its first k-blocks, which finishes it) and tail (its last
- * k-blocks, whose int32 sums are handed over) sit in adjacent pairs.
+ * pairs under split mode `mode` (INT8LT_SPLIT_*), as the kernel walks it.
+ * Writes up to cap_rows rows of 6 int32 (pair, tile, first k-block, end
+ * k-block, head flag, tail flag) and returns the number of segments (or -1
+ * for bad arguments). A split tile's head (its first k-blocks, which finishes
+ * it) and tail (its last k-blocks, whose int32 sums are handed over) sit in
+ * adjacent pairs.
  */
-int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int32_t *out, int cap_rows);
+int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int mode, int32_t *out, int cap_rows);
 
 /*
  * Test entry: launch one block that waits on a barrier nothing ever arrives

@@ -19,10 +19,10 @@ def L():
     return _lib.lib()
 
 
-def schedule(L, tiles, nkb, pairs):
-    n = L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, None, 0)
+def schedule(L, tiles, nkb, pairs, mode=_lib.SPLIT_ALWAYS):
+    n = L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, mode, None, 0)
     out = np.zeros((max(n, 1), 6), np.int32)
-    assert L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, out.ctypes.data, n) == n
+    assert L.int8lt_debug_gemm_schedule(tiles, nkb, pairs, mode, out.ctypes.data, n) == n
     return out[:n]
 
 
@@ -69,5 +69,38 @@ def test_schedule_covers_every_kblock_once(L, tiles, nkb, pairs):
 
 
 def test_bad_arguments(L):
-    assert L.int8lt_debug_gemm_schedule(4, 0, 2, None, 0) == -1
-    assert L.int8lt_debug_gemm_schedule(4, 2, 0, None, 0) == -1
+    assert L.int8lt_debug_gemm_schedule(4, 0, 2, 0, None, 0) == -1
+    assert L.int8lt_debug_gemm_schedule(4, 2, 0, 0, None, 0) == -1
+    assert L.int8lt_debug_gemm_schedule(4, 2, 2, 3, None, 0) == -1
+
+
+def _is_split(s):
+    return bool(s[:, 5].any())
+
+
+@pytest.mark.parametrize("tiles,nkb,pairs,want", [
+    (76, 64, 74, True),     # 1024 x 4864 x 8192: 1.03 waves, the second nearly empty
+    (256, 128, 74, True),   # 4096 x 4096 x 16384: saves 69 k-blocks per pair
+    (128, 32, 74, False),   # 2048 x 4096 x 4096: saves under 9 k-blocks per pair
+    (80, 32, 74, False),    # saves 29 k-blocks, below one 4096-deep tile
+    (1024, 32, 74, False),
+    (148, 32, 74, False),   # exact waves: nothing to split
+])
+def test_auto_policy(L, tiles, nkb, pairs, want):
+    assert _is_split(schedule(L, tiles, nkb, pairs, _lib.SPLIT_AUTO)) == want
+    assert not _is_split(schedule(L, tiles, nkb, pairs, _lib.SPLIT_NEVER))
+    s_auto = schedule(L, tiles, nkb, pairs, _lib.SPLIT_AUTO)
+    cover = np.zeros((tiles, nkb), np.int32)
+    for p, t, k0, k1, h, tl in s_auto:
+        cover[t, k0:k1] += 1
+    assert (cover == 1).all()
+
+
+def test_set_gemm_split_roundtrip(L):
+    prev = _lib.int8lt_set_gemm_split(_lib.SPLIT_NEVER)
+    try:
+        assert _lib.int8lt_set_gemm_split(_lib.SPLIT_ALWAYS) == _lib.SPLIT_NEVER
+        with pytest.raises(ValueError):
+            _lib.int8lt_set_gemm_split(7)
+    finally:
+        _lib.int8lt_set_gemm_split(prev)

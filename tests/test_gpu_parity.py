@@ -112,13 +112,31 @@ def test_gemm_int32_bit_exact(M, N, K):
 SPLIT_SHAPES = [(1280, 4096, 512), (2048, 4096, 384), (2304, 4352, 1152)]
 
 
+@pytest.fixture
+def split_always():
+    prev = _lib.int8lt_set_gemm_split(_lib.SPLIT_ALWAYS)
+    yield
+    _lib.int8lt_set_gemm_split(prev)
+
+
 @pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
-def test_gemm_int32_split_tiles_bit_exact(M, N, K):
+def test_gemm_int32_split_tiles_bit_exact(M, N, K, split_always):
     rng = np.random.default_rng(M + N + K)
     A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
     B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
     C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
     assert np.array_equal(C, oracle.gemm_i32(A, B))
+
+
+def test_gemm_int32_split_auto_sampled_rows():
+    # 4 x 19 = 76 tiles of 64 k-blocks: the default policy splits the last wave
+    M, N, K = 1024, 4864, 8192
+    rng = np.random.default_rng(76)
+    A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    rows = np.array([0, 1, 255, 256, 300, 511, 512, 700, 767, 768, 1000, 1023])
+    assert np.array_equal(C[rows], oracle.gemm_i32(A[rows], B))
 
 
 def test_gemm_int32_matches_oracle_routine():
@@ -169,9 +187,17 @@ SPLIT_FCASES = [
 
 
 @pytest.mark.parametrize("w", SPLIT_FCASES, ids=[w.name for w in SPLIT_FCASES])
-def test_forward_split_tiles_vs_oracle(w):
+def test_forward_split_tiles_vs_oracle(w, split_always):
     X, W, b = case_inputs(w)
     Yg, Y64 = run_forward(X, W, b, w.threshold)
+    check_y(Yg, Y64, w.name)
+
+
+def test_forward_split_auto_sampled_rows():
+    w = wl.random_case(62, 1024, 8192, 4864, n_outliers=6, frac=0.5)
+    X, W, b = case_inputs(w)
+    rows = [0, 1, 255, 256, 511, 512, 767, 768, 900, 1023]
+    Yg, Y64 = run_forward(X, W, b, w.threshold, rows=rows)
     check_y(Yg, Y64, w.name)
 
 
