@@ -397,6 +397,42 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
             }
         }
     }
+    // Outlier-weight gather Wo[j, t] = W[j, col_t] (or CB[j, col_t] * SCB[j]
+    // / 127): half-warps over output channels, a lane per outlier rank t,
+    // four channels per pass. The first pass's loads are issued before phase
+    // B and stored after it, so their latency hides behind the quantization.
+    const int hl = lane & 15;
+    const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
+    const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
+    __half gv[4];
+    auto gather_load = [&](int32_t t0, int64_t j0) {
+        const int32_t t = t0 + hl;
+        const bool real = t < n_out;
+        const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t j = j0 + u * nhw;
+            gv[u] = __float2half_rn(0.f);
+            if (real && j < a.N) {
+                if (a.W_outlier) {
+                    gv[u] = a.W_outlier[j * a.K + col];
+                } else {
+                    const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
+                    gv[u] = __float2half_rn(__fdiv_rn(p, 127.f));
+                }
+            }
+        }
+    };
+    auto gather_store = [&](int32_t t0, int64_t j0) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t j = j0 + u * nhw;
+            if (j < a.N) a.Wo[j * a.kcap + t0 + hl] = gv[u];
+        }
+    };
+    const bool gather = a.Wo && n16 > 0;
+    if (gather) gather_load(0, hw);
+
     for (int rd = rounds - 1; rd >= 0; --rd) {
         const int64_t r0 = ((int64_t)rd * gridDim.x + blockIdx.x) * rows_per_round;
         const int64_t left = a.M - r0;
@@ -424,38 +460,13 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
             }
         }
     }
-    if (a.Wo) {
-        // Wo[j, t] = W[j, col_t]: half-warps over output channels, a lane per
-        // outlier rank t, four channels' loads in flight before any store.
-        const int hl = lane & 15;
-        const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
-        const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
-        for (int32_t t0 = 0; t0 < n16; t0 += 16) {
-            const int32_t t = t0 + hl;
-            const bool real = t < n_out;
-            const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
-            for (int64_t j0 = hw; j0 < a.N; j0 += 4 * nhw) {
-                __half val[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t j = j0 + u * nhw;
-                    val[u] = __float2half_rn(0.f);
-                    if (real && j < a.N) {
-                        if (a.W_outlier) {
-                            val[u] = a.W_outlier[j * a.K + col];
-                        } else {
-                            const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
-                            val[u] = __float2half_rn(__fdiv_rn(p, 127.f));
-                        }
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t j = j0 + u * nhw;
-                    if (j < a.N) a.Wo[j * a.kcap + t] = val[u];
-                }
+    if (gather) {
+        gather_store(0, hw);
+        for (int32_t t0 = 0; t0 < n16; t0 += 16)
+            for (int64_t j0 = hw + (t0 == 0 ? 4 * nhw : 0); j0 < a.N; j0 += 4 * nhw) {
+                gather_load(t0, j0);
+                gather_store(t0, j0);
             }
-        }
     }
     const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x, nth = (int64_t)gridDim.x * kThreads;
     if (a.acc)
