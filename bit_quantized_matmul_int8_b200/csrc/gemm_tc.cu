@@ -115,7 +115,10 @@ constexpr uint32_t kTxBytes = 2 * (kStageA + kStageB);  // both CTAs, counted by
 constexpr int kOkb = 32;                  // outlier columns per k-block (64-byte rows)
 constexpr int kOStage = kCtaRows * kOkb * 2;            // bytes of Xo (or Wo) per CTA: 8 KB
 constexpr uint32_t kOTxBytes = 2 * 2 * kOStage;         // Xo + Wo of both CTAs
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 8;                      // 2 per TMEM lane quadrant
+constexpr int kEpiCols = BN * 4 / kEpiWarps;      // accumulator columns per epilogue warp
+constexpr int kEpiChunks = kEpiCols / 32;         // tcgen05.ld chunks of 32 columns per warp
+constexpr int kBoxes = 2;                         // fp16 store boxes per epilogue warp
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
@@ -150,8 +153,8 @@ constexpr int kStoreBox = 32;                                    // Y staged in 
 constexpr size_t kStoreBufBytes = kStoreBox * kStoreBox * 2;     // 2 KB
 constexpr size_t kSmemTiles = (size_t)kStages * (kStageA + kStageB);
 constexpr size_t kOffOut = kSmemTiles;                           // Xo slot, then Wo slot
-constexpr size_t kOffStage = kOffOut + 2 * (size_t)kOStage;      // [kEpiWarps][2] store boxes
-constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * 2 * kStoreBufBytes;
+constexpr size_t kOffStage = kOffOut + 2 * (size_t)kOStage;      // [kEpiWarps][kBoxes] store boxes
+constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * kBoxes * kStoreBufBytes;
 constexpr size_t kOffScb = kOffCtrl + 256;
 constexpr size_t kOffBias = kOffScb + BN * 4;
 constexpr size_t kSmemUsed = kOffBias + BN * 4;
@@ -179,18 +182,18 @@ __device__ __forceinline__ void arrive_leader(Ctrl *ctrl, uint64_t *bar, uint32_
 
 // Partial sums of a split tile's tail, written so that each store of a
 // warp covers 512 contiguous bytes: int4 (v) of chunk cc of lane l of
-// epilogue warp ew sits at slot[((ew * 4 + cc / 32) * 8 + v) * 32 + l]. The
+// epilogue warp ew sits at slot[((ew * kEpiChunks + cc / 32) * 8 + v) * 32 + l]. The
 // head reads them back with the same warp and lane, which own the same rows
 // and columns in both CTAs' epilogues.
 __device__ __forceinline__ void epilogue_store_partial(uint32_t tmem, uint32_t lane_base, int buf, int hcol, int ew,
                                                        int lane, uint32_t rank, Ctrl *ctrl, int4 *slot) {
-    const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
-    int4 *dst = slot + (size_t)ew * 4 * 8 * 32 + lane;
-    for (int cc = 0; cc < 128; cc += 32) {
+    const uint32_t col0 = (uint32_t)(buf * 256 + hcol * kEpiCols);
+    int4 *dst = slot + (size_t)ew * kEpiChunks * 8 * 32 + lane;
+    for (int cc = 0; cc < kEpiCols; cc += 32) {
         uint32_t acc[32];
         tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
         tmem_ld_wait();
-        if (cc == 96) {
+        if (cc == kEpiCols - 32) {
             tc_fence_before();
             if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
         }
@@ -250,9 +253,12 @@ __device__ __forceinline__ void store32(const uint32_t (&y)[32], uint8_t *s_stag
         __half2 h = __float22half2_rn(make_float2(__uint_as_float(y[2 * k]), __uint_as_float(y[2 * k + 1])));
         packed[k] = *reinterpret_cast<uint32_t *>(&h);
     }
-    if (lane == 0) bulk_wait_read_1();  // this box's previous store has read it
+    if (lane == 0) {  // this box's previous store has read it
+        if constexpr (kBoxes == 2) bulk_wait_read_1();
+        else bulk_wait_read_0();
+    }
     __syncwarp();
-    uint8_t *box = s_stage + (size_t)(ew * 2 + sbuf) * kStoreBufBytes;
+    uint8_t *box = s_stage + (size_t)(ew * kBoxes + sbuf) * kStoreBufBytes;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         *reinterpret_cast<uint4 *>(box + lane * 64 + ((i ^ ((lane >> 1) & 3)) * 16)) =
@@ -263,7 +269,7 @@ __device__ __forceinline__ void store32(const uint32_t (&y)[32], uint8_t *s_stag
         tma_store_2d(tmY, smem_u32(box), x, yrow);
         bulk_commit_group();
     }
-    sbuf ^= 1;
+    sbuf = kBoxes == 2 ? sbuf ^ 1 : 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -524,8 +530,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // ---------------------------------------------------- epilogue --
         const int ew = warp - 2;                 // 0..7
         const int q = warp & 3;                  // TMEM lanes [32q, 32q + 32) are this warp's
-        const int hcol = ew >> 2;                // columns [128 hcol, 128 hcol + 128)
-        const int et = threadIdx.x - 64;         // 0..255
+        const int hcol = ew >> 2;                // columns [kEpiCols hcol, kEpiCols (hcol + 1))
+        const int et = threadIdx.x - 64;         // 0 .. kEpiThreads - 1; thread et < BN stages column et
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         int sbuf = 0;  // which of the warp's two store boxes is next
         int it = 0;
@@ -540,7 +546,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // Fetch this tile's column data (thread et owns column n0 + et)
             // and this thread's row scale while the MMAs are still running.
             const int64_t col = n0 + et;
-            const bool col_ok = !a.C32 && col < a.N;
+            const bool col_ok = !a.C32 && et < BN && col < a.N;
             const float scb_v = col_ok ? a.SCB[col] : 0.f;
             const float bias_v = (col_ok && a.bias) ? __half2float(a.bias[col]) : 0.f;
             const int64_t row = m0 + q * 32 + lane;
@@ -560,13 +566,13 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 *abort_flag = 1;
                 break;
             }
-            if (!a.C32) {
+            if (!a.C32 && et < BN) {
                 s_scb[et] = scb_v;
                 s_bias[et] = bias_v;
             }
             epi_sync();
             tc_fence_after();
-            const uint32_t col0 = (uint32_t)(buf * 256 + hcol * 128);
+            const uint32_t col0 = (uint32_t)(buf * 256 + hcol * kEpiCols);
             if (g.tail) {
                 // Tail of a split tile: hand the int32 sums to the head's pair.
                 int4 *slot = reinterpret_cast<int4 *>(a.sk_partial) + (size_t)(pair * 2 + rank) * (kSkPartialBytes / 16);
@@ -592,21 +598,21 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 epi_sync();
                 part = reinterpret_cast<const int4 *>(a.sk_partial) +
-                       (size_t)((pair + 1) * 2 + rank) * (kSkPartialBytes / 16) + (size_t)ew * 4 * 8 * 32 + lane;
+                       (size_t)((pair + 1) * 2 + rank) * (kSkPartialBytes / 16) + (size_t)ew * kEpiChunks * 8 * 32 + lane;
             }
             const float rs = sca_v * (1.0f / 16129.0f);
             if (a.C32) {
                 // Raw int32 sums (test entry): no scales, no outliers.
-                for (int cc = 0; cc < 128; cc += 32) {
+                for (int cc = 0; cc < kEpiCols; cc += 32) {
                     uint32_t acc[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
                     tmem_ld_wait();
-                    if (cc == 96) {
+                    if (cc == kEpiCols - 32) {
                         tc_fence_before();
                         if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
                     }
                     add_partial(acc, part, cc);
-                    const int64_t c0 = n0 + hcol * 128 + cc;
+                    const int64_t c0 = n0 + hcol * kEpiCols + cc;
                     if (!row_ok || c0 >= a.N) continue;
                     int32_t *dst = a.C32 + row * a.N + c0;
 #pragma unroll
@@ -617,11 +623,11 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
             } else if (n_okb) {
                 // Pass 1: fp32 C * rs * SCB + bias back into the buffer.
-                for (int cc = 0; cc < 128; cc += 32) {
+                for (int cc = 0; cc < kEpiCols; cc += 32) {
                     uint32_t acc[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
                     tmem_ld_wait();
-                    dequant32(acc, rs, s_scb + hcol * 128 + cc, s_bias + hcol * 128 + cc, part, cc);
+                    dequant32(acc, rs, s_scb + hcol * kEpiCols + cc, s_bias + hcol * kEpiCols + cc, part, cc);
                     tmem_st_32x32b_x32(tmem + lane_base + col0 + cc, acc);
                 }
                 tmem_st_wait();
@@ -640,31 +646,31 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 tc_fence_after();
                 // Pass 2: fp16 out.
-                for (int cc = 0; cc < 128; cc += 32) {
+                for (int cc = 0; cc < kEpiCols; cc += 32) {
                     uint32_t y[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, y);
                     tmem_ld_wait();
-                    if (cc == 96) {
+                    if (cc == kEpiCols - 32) {
                         tc_fence_before();
                         if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
                     }
-                    if (n0 + hcol * 128 + cc < a.N)
-                        store32(y, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * 128 + cc),
+                    if (n0 + hcol * kEpiCols + cc < a.N)
+                        store32(y, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * kEpiCols + cc),
                                 (int32_t)(m0 + q * 32));
                 }
             } else {
                 // No outliers: one pass.
-                for (int cc = 0; cc < 128; cc += 32) {
+                for (int cc = 0; cc < kEpiCols; cc += 32) {
                     uint32_t acc[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + col0 + cc, acc);
                     tmem_ld_wait();
-                    if (cc == 96) {
+                    if (cc == kEpiCols - 32) {
                         tc_fence_before();
                         if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
                     }
-                    if (n0 + hcol * 128 + cc >= a.N) continue;  // whole chunk past the last column
-                    dequant32(acc, rs, s_scb + hcol * 128 + cc, s_bias + hcol * 128 + cc, part, cc);
-                    store32(acc, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * 128 + cc),
+                    if (n0 + hcol * kEpiCols + cc >= a.N) continue;  // whole chunk past the last column
+                    dequant32(acc, rs, s_scb + hcol * kEpiCols + cc, s_bias + hcol * kEpiCols + cc, part, cc);
+                    store32(acc, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * kEpiCols + cc),
                             (int32_t)(m0 + q * 32));
                 }
             }

@@ -264,6 +264,29 @@ __device__ __forceinline__ void quantize_row_plain(const QuantizeArgs &a, const 
     if (lane == 0) a.SCA[r] = sa;
 }
 
+// Phase B of a long staged row (outlier elements already zero) by the whole
+// CTA; every thread calls it. s_red holds one maximum per warp.
+__device__ __forceinline__ void quantize_row_cta(const QuantizeArgs &a, const uint4 *row, int64_t r, uint32_t *s_red,
+                                                 int lane, int warp) {
+    const int nvec = (int)(a.K / 8);
+    uint32_t m = 0;
+#pragma unroll 4
+    for (int v = threadIdx.x; v < nvec; v += kThreads) m = max(m, vec_absmax_bits(row[v]));
+    m = warp_max_u32(m);
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    uint32_t amax = s_red[0];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) amax = max(amax, s_red[i]);
+    const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+    const float s = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+    uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+#pragma unroll 4
+    for (int v = threadIdx.x; v < nvec; v += kThreads) ca2[v] = quant_vec8(row[v], s);
+    if (threadIdx.x == 0) a.SCA[r] = sa;
+    __syncthreads();  // s_red is free again
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -308,19 +331,21 @@ __device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base) {
 // Phase A walks the CTA's rows in rounds of R rows (rows of a round are
 // contiguous in X): every thread keeps 16 16-byte loads in flight, tests
 // them and, in the last round, also keeps them in shared memory. Phase B
-// quantizes the last round from shared memory and the earlier rounds from X
-// again (from L2 when X fits); with a single round X is read from HBM
-// exactly once. R = 0 (rows too long to keep): phase B reads every row from X.
+// quantizes the last round from shared memory, then brings each earlier
+// round back into shared memory (from L2 when X fits) and does the same; with
+// a single round X is read from HBM exactly once. R = 0 (rows too long to
+// keep): phase B reads every row from X, a warp per row.
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
     extern __shared__ __align__(128) uint32_t smem[];
-    __shared__ uint32_t s_gen, s_base;
+    __shared__ uint32_t s_gen, s_base, s_red[kWarps];
     uint32_t *bits = smem;                                         // [kwords]
     int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
     uint4 *rows = reinterpret_cast<uint4 *>(smem + ((2 * kwords + 31) & ~int64_t(31)));  // [R][nvec]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nvec = (int)(a.K / 8);
     const int rows_per_round = R > 0 ? R : kWarps;
+    const bool long_rows = nvec >= 4 * kThreads;  // K >= 8192: a CTA per staged row
     const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
     const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
     // The GEMM behind this pass may start its prologue on SMs this grid frees;
@@ -437,27 +462,52 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
         const int64_t r0 = ((int64_t)rd * gridDim.x + blockIdx.x) * rows_per_round;
         const int64_t left = a.M - r0;
         const int nr = left <= 0 ? 0 : (left < rows_per_round ? (int)left : rows_per_round);
-        for (int r = warp; r < nr; r += kWarps) {
-            if (R > 0 && rd == rounds - 1) {
-                // Staged row: copy its outlier elements to Xo and zero them
-                // in place, then quantize it without masks.
-                uint4 *row = rows + (size_t)r * nvec;
-                __half *rh = reinterpret_cast<__half *>(row);
-                __half *xo = a.Xo ? a.Xo + (r0 + r) * a.kcap : nullptr;
-                for (int32_t t = lane; t < n16; t += 32) {
-                    __half val = __float2half_rn(0.f);
-                    if (t < n_out) {
-                        const int64_t col = outlier_column(bits, prefix, kwords, t);
-                        val = rh[col];
-                        rh[col] = __ushort_as_half((unsigned short)0);
-                    }
-                    if (xo) xo[t] = val;
-                }
-                __syncwarp();
-                quantize_row_plain(a, row, r0 + r, lane);
-            } else {
+        if (R == 0) {
+            for (int r = warp; r < nr; r += kWarps)
                 quantize_row<false>(a, X4 + (r0 + r) * nvec, r0 + r, bits, prefix, n_out, lane);
+            continue;
+        }
+        if (rd != rounds - 1) {
+            // An earlier round: bring its rows back into shared memory.
+            __syncthreads();  // the previous round's rows are done with
+            const int64_t total = (int64_t)nr * nvec;
+            const uint4 *src = X4 + r0 * nvec;
+            for (int64_t flat = threadIdx.x; flat < total; flat += kBatch * kThreads) {
+                uint4 x[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int64_t f = flat + u * kThreads;
+                    x[u] = f < total ? __ldg(src + f) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int64_t f = flat + u * kThreads;
+                    if (f < total) rows[f] = x[u];
+                }
             }
+            __syncthreads();
+        }
+        // Staged rows: copy their outlier elements to Xo and zero them in
+        // place (a warp per row), then quantize them without masks: a warp
+        // per row, or the whole CTA per row when rows are long.
+        for (int r = warp; r < nr; r += kWarps) {
+            __half *rh = reinterpret_cast<__half *>(rows + (size_t)r * nvec);
+            __half *xo = a.Xo ? a.Xo + (r0 + r) * a.kcap : nullptr;
+            for (int32_t t = lane; t < n16; t += 32) {
+                __half val = __float2half_rn(0.f);
+                if (t < n_out) {
+                    const int64_t col = outlier_column(bits, prefix, kwords, t);
+                    val = rh[col];
+                    rh[col] = __ushort_as_half((unsigned short)0);
+                }
+                if (xo) xo[t] = val;
+            }
+            __syncwarp();
+            if (!long_rows) quantize_row_plain(a, rows + (size_t)r * nvec, r0 + r, lane);
+        }
+        if (long_rows) {
+            __syncthreads();
+            for (int r = 0; r < nr; ++r) quantize_row_cta(a, rows + (size_t)r * nvec, r0 + r, s_red, lane, warp);
         }
     }
     if (gather) {
@@ -567,8 +617,11 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
         if (cudaError_t e = quant_resident((int)bits_bytes, &resident)) return e;
         if (resident <= 0) return cudaErrorInvalidConfiguration;
         grid = (int)std::min<int64_t>(resident, std::max<int64_t>(1, ceil_div(a.M, kWarps)));
-        rounds = (int)ceil_div(a.M, (int64_t)kWarps * grid);  // kWarps rows per CTA and round
     }
+    // The outlier-weight gather and the split-K clears run over all N output
+    // channels: give them enough CTAs even when there are few rows.
+    if (a.Wo || a.acc) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.N, 32)));
+    if (R == 0) rounds = (int)ceil_div(a.M, (int64_t)kWarps * grid);  // kWarps rows per CTA and round
     // The grid barrier needs every CTA resident at once: a cooperative launch.
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];

@@ -51,6 +51,12 @@ QCASES = [
     ("wide", wl.random_case(42, 130, 4112, 8, n_outliers=9, frac=0.75), None),
     ("many_rows", wl.random_case(43, 3000, 256, 8, n_outliers=3, frac=0.01), None),
     ("no_outliers", wl.random_case(44, 64, 512, 8, n_outliers=0), None),
+    # more rows than shared memory keeps at once: several rounds
+    ("rounds", wl.random_case(45, 4000, 4096, 8, n_outliers=7, frac=0.5), None),
+    # rows of K >= 8192 are quantized by a whole CTA each, in rounds
+    ("long_rows", wl.random_case(46, 1000, 16384, 8, n_outliers=4, frac=0.75), None),
+    # rows too long to keep in shared memory: read from X in both phases
+    ("very_long_rows", wl.random_case(47, 20, 65536, 8, n_outliers=3, frac=0.5), None),
 ]
 
 
