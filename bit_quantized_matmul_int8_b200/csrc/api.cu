@@ -30,8 +30,8 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
     } else {
         L.wo = SIZE_MAX;
         L.sk = SIZE_MAX;
-        L.acc = off; off += align_up((size_t)N * 16 * 4);
-        L.cnt = off; off += align_up((size_t)ceil_div(N, 32) * 4);
+        L.acc = off; off += align_up((size_t)round_up(N * M, 4) * 4);
+        L.cnt = off; off += align_up((size_t)round_up(ceil_div(N, 8), 4) * 4);
     }
     L.total = off;
     return L;
@@ -122,7 +122,6 @@ int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_
     const __half *x = static_cast<const __half *>(X);
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
     const bool decode = M <= kDecodeMaxM;
-    const int splits = decode ? gemv_splits(N, K) : 1;
     QuantizeArgs q{};
     q.X = x; q.M = M; q.K = K;
     q.hdr = hdr; q.bitmaps = at<uint32_t>(ws, L.bitmaps); q.tbits = threshold_bits(threshold);
@@ -131,9 +130,9 @@ int forward_quantize(const void *X, int64_t M, int64_t N, int64_t K, const int8_
     q.Xo = at<__half>(ws, L.xo); q.kcap = L.kcap;
     q.W_outlier = static_cast<const __half *>(W_outlier); q.CB = CB; q.SCB = SCB; q.N = N;
     if (!decode) q.Wo = at<__half>(ws, L.wo);
-    if (decode && splits > 1) {
-        q.acc = at<int32_t>(ws, L.acc); q.acc_words = N * 16;
-        q.cnt = at<uint32_t>(ws, L.cnt); q.cnt_words = ceil_div(N, 32);
+    if (decode) {  // the GEMV's partial sums and k-block counters start at zero
+        q.acc = at<int32_t>(ws, L.acc); q.acc_words = round_up(N * M, 4);
+        q.cnt = at<uint32_t>(ws, L.cnt); q.cnt_words = round_up(ceil_div(N, 8), 4);
     }
     return from_cuda(launch_quantize(q, s));
 }
@@ -143,15 +142,14 @@ int forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const floa
     const WsLayout L = ws_layout(M, N, K);
     WsHeader *hdr = at<WsHeader>(ws, L.hdr);
     if (M <= kDecodeMaxM) {
-        const int splits = gemv_splits(N, K);
         GemvArgs g{};
         g.CA = at<int8_t>(ws, L.ca); g.CB = CB; g.SCA = at<float>(ws, L.sca); g.SCB = SCB;
         g.Xo = at<__half>(ws, L.xo); g.kcap = L.kcap;
         g.outlier_idx = at<int32_t>(ws, L.idx); g.n_outliers = &hdr->n_outliers;
         g.W_outlier = static_cast<const __half *>(W_outlier); g.bias = static_cast<const __half *>(bias);
         g.Y = static_cast<__half *>(Y);
-        if (splits > 1) { g.acc = at<int32_t>(ws, L.acc); g.cnt = at<uint32_t>(ws, L.cnt); }
-        g.M = M; g.N = N; g.K = K; g.splits = splits;
+        g.acc = at<int32_t>(ws, L.acc); g.cnt = at<uint32_t>(ws, L.cnt); g.status = &hdr->status;
+        g.M = M; g.N = N; g.K = K;
         return from_cuda(launch_gemv(g, s));
     }
     GemmArgs g{};
@@ -196,9 +194,10 @@ int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream) {
     if (!ws) return INT8LT_ERR_NULL;
     if (ws_bytes < sizeof(WsHeader)) return INT8LT_ERR_WORKSPACE;
     if (!aligned(ws, 16)) return INT8LT_ERR_ALIGN;
-    // header (status, outlier count, quantize generation and barrier count)
-    // and both column bitmaps
-    return from_cuda(cudaMemsetAsync(ws, 0, std::min(ws_bytes, kWsInitBytes), static_cast<cudaStream_t>(stream)));
+    // Everything, so that the header (status, outlier count, quantize
+    // generation and barrier counts), both column bitmaps and the split-tile
+    // flags start at zero; later calls keep them consistent.
+    return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream) {
@@ -292,14 +291,12 @@ int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t
     if (M <= kDecodeMaxM) {
         GemvArgs g{};
         g.CA = CA; g.CB = CB; g.C32 = C;
-        g.M = M; g.N = N; g.K = K; g.splits = gemv_splits(N, K);
-        if (g.splits > 1) {
-            g.acc = at<int32_t>(ws, L.acc);
-            g.cnt = at<uint32_t>(ws, L.cnt);
-            if (cudaMemsetAsync(g.acc, 0, (size_t)N * 16 * 4, s) != cudaSuccess ||
-                cudaMemsetAsync(g.cnt, 0, (size_t)ceil_div(N, 32) * 4, s) != cudaSuccess)
-                return INT8LT_ERR_CUDA;
-        }
+        g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+        g.acc = at<int32_t>(ws, L.acc);
+        g.cnt = at<uint32_t>(ws, L.cnt);
+        if (cudaMemsetAsync(g.acc, 0, (size_t)N * M * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(g.cnt, 0, (size_t)ceil_div(N, 8) * 4, s) != cudaSuccess)
+            return INT8LT_ERR_CUDA;
         return from_cuda(launch_gemv(g, s));
     }
     GemmArgs g{};

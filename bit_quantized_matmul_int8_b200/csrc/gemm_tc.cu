@@ -693,8 +693,11 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
+}  // namespace
+
 // ----------------------------------------------------------- tensor maps --
 
+namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -713,13 +716,10 @@ EncodeTiledFn get_encode_fn() {
     });
     return fn;
 }
+}  // namespace
 
-// 2-D row-major map: `inner` elements per row (contiguous), `outer` rows,
-// row pitch `pitch_bytes`; box of box_inner x box_outer; 128-byte swizzle;
-// out-of-range elements read as zero.
 bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
-              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -731,6 +731,7 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
 int g_num_sms[64];  // resident CTA pairs per device
 
 }  // namespace

@@ -15,7 +15,16 @@
 //     used as they lie, with the same permutation applied to A and B;
 //   - K is split across warps when N alone gives too few warps; the int32
 //     partial sums are added with atomics (exact in any order) and the last
-//     warp of a row group, found with an arrival counter, runs the epilogue.
+//     warp of a row group, found with an arrival counter, runs the epilogue
+//     (the quantize pass zeroes the sums and the counters);
+//   - launched with programmatic stream serialization, each warp starts
+//     pulling the first kilobyte of its weight rows into L2 before it waits
+//     for the quantize pass.
+// Each warp reads 32 rows 128 bytes at a time. A read-bandwidth probe on
+// this pool put that pattern at about 4.2-4.9 TB/s against 6.5-6.8 TB/s for
+// reads of 1 KB or more per row; designs that stream longer pieces per row
+// (TMA boxes of 64 rows x 128 bytes issued eight at a time, per-row 1 KB
+// bulk copies) measured slower here, so this one stays.
 #include <algorithm>
 
 #include "int8lt_internal.cuh"
@@ -27,6 +36,15 @@ namespace {
 constexpr int kWarpsPerCta = 8;
 constexpr int kRowsPerWarp = 32;
 constexpr int kTargetWarps = 148 * 8;
+constexpr int kHalves = 2;  // 64-byte pieces of K per row per step (the step is kHalves * 64 bytes)
+
+// Warps that share the K range of one row group (1 = none).
+int gemv_splits(int64_t N, int64_t K) {
+    const int64_t rg = ceil_div(N, kRowsPerWarp);
+    int64_t s = ceil_div(kTargetWarps, rg);
+    s = std::min<int64_t>(s, std::max<int64_t>(1, K / 256));
+    return (int)std::max<int64_t>(1, std::min<int64_t>(s, 64));
+}
 
 __device__ __forceinline__ void mma_16832_s8(int32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -62,16 +80,29 @@ __device__ __forceinline__ void finish(const GemvArgs &a, int n_out, int64_t t, 
 }
 
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
-gemv_i8_kernel(const GemvArgs a, const int64_t row_groups) {
+gemv_i8_kernel(const GemvArgs a, const int64_t row_groups, const int splits) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, tig = lane & 3;
     const int64_t unit = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-    if (unit >= row_groups * a.splits) return;
-    const int64_t rg = unit / a.splits;
-    const int sp = (int)(unit % a.splits);
+    if (unit >= row_groups * splits) return;
+    const int64_t rg = unit / splits;
+    const int sp = (int)(unit % splits);
     const int64_t n0 = rg * kRowsPerWarp;
-    const int64_t kchunk = round_up(ceil_div(a.K, a.splits), 64);
+    const int64_t kchunk = round_up(ceil_div(a.K, splits), 64);
     const int64_t k0 = sp * kchunk, k1 = min(a.K, k0 + kchunk);
+
+    // Until the quantize pass before this kernel has finished, only CB (which
+    // it does not write) may be touched: pull the first kilobyte of each of
+    // this warp's 32 weight rows into L2, then wait.
+    {
+        const int64_t j = n0 + lane;
+        if (j < a.N && k0 < k1) {
+            const uint32_t bytes = (uint32_t)(k1 - k0 < 1024 ? k1 - k0 : 1024);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.CB + j * a.K + k0), "r"(bytes)
+                         : "memory");
+        }
+    }
+    grid_dep_wait();
 
     const bool tok_lo = g < a.M, tok_hi = g + 8 < a.M;
     const int8_t *xa = a.CA + (int64_t)g * a.K;
@@ -90,10 +121,10 @@ gemv_i8_kernel(const GemvArgs a, const int64_t row_groups) {
     for (int q = 0; q < 4; ++q) d[q][0] = d[q][1] = d[q][2] = d[q][3] = 0;
 
     const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int64_t k = k0; k < k1; k += 128) {
-        uint4 w[2][4], xl[2], xh[2];
+    for (int64_t k = k0; k < k1; k += kHalves * 64) {
+        uint4 w[kHalves][4], xl[kHalves], xh[kHalves];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kHalves; ++h) {
             const int64_t kk = k + h * 64 + tig * 16;
             const bool kin = kk < k1;
 #pragma unroll
@@ -102,7 +133,7 @@ gemv_i8_kernel(const GemvArgs a, const int64_t row_groups) {
             xh[h] = (kin && tok_hi) ? __ldg(reinterpret_cast<const uint4 *>(xb + kk)) : z;
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kHalves; ++h) {
             const uint32_t a0[4] = {xl[h].x, xh[h].x, xl[h].y, xh[h].y};
             const uint32_t a1[4] = {xl[h].z, xh[h].z, xl[h].w, xh[h].w};
 #pragma unroll
@@ -115,26 +146,26 @@ gemv_i8_kernel(const GemvArgs a, const int64_t row_groups) {
 
     // Fragment owner: d[q][0..1] -> token g, channels n0 + 8q + 2tig + {0,1};
     //                 d[q][2..3] -> token g + 8, same channels.
-    if (a.splits > 1) {
+    if (splits > 1) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int64_t t = g + (e >> 1) * 8, j = n0 + 8 * q + 2 * tig + (e & 1);
-                if (t < a.M && j < a.N) atomicAdd(&a.acc[j * 16 + t], d[q][e]);
+                if (t < a.M && j < a.N) atomicAdd(&a.acc[j * a.M + t], d[q][e]);
             }
         __threadfence();
         uint32_t old = 0;
         if (lane == 0) old = atomicAdd(&a.cnt[rg], 1u);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != (uint32_t)a.splits - 1) return;
+        if (old != (uint32_t)splits - 1) return;
         __threadfence();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int64_t t = g + (e >> 1) * 8, j = n0 + 8 * q + 2 * tig + (e & 1);
-                d[q][e] = (t < a.M && j < a.N) ? __ldcg(&a.acc[j * 16 + t]) : 0;
+                d[q][e] = (t < a.M && j < a.N) ? __ldcg(&a.acc[j * a.M + t]) : 0;
             }
     }
 
@@ -159,18 +190,20 @@ gemv_i8_kernel(const GemvArgs a, const int64_t row_groups) {
 
 }  // namespace
 
-int gemv_splits(int64_t N, int64_t K) {
-    const int64_t rg = ceil_div(N, kRowsPerWarp);
-    int64_t s = ceil_div(kTargetWarps, rg);
-    s = std::min<int64_t>(s, std::max<int64_t>(1, K / 256));
-    return (int)std::max<int64_t>(1, std::min<int64_t>(s, 64));
-}
-
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s) {
     const int64_t rg = ceil_div(a.N, kRowsPerWarp);
-    const int64_t warps = rg * a.splits;
-    gemv_i8_kernel<<<(unsigned)ceil_div(warps, kWarpsPerCta), kWarpsPerCta * 32, 0, s>>>(a, rg);
-    return cudaGetLastError();
+    const int splits = gemv_splits(a.N, a.K);
+    const int64_t warps = rg * splits;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)ceil_div(warps, kWarpsPerCta), 1, 1);
+    cfg.blockDim = dim3(kWarpsPerCta * 32, 1, 1);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_i8_kernel, a, rg, splits);
 }
 
 }  // namespace int8lt

@@ -77,9 +77,9 @@ struct QuantizeArgs {
     const float *SCB;
     __half *Wo;               // [N][kcap] or null (no gather)
     int64_t N;
-    // Split-K reduction buffers to clear (M <= 16 path), or null.
+    // Decode path: partial-sum buffers to zero for the GEMV, or null.
     int32_t *acc;
-    int64_t acc_words;
+    int64_t acc_words;        // a multiple of 4
     uint32_t *cnt;
     int64_t cnt_words;
 };
@@ -120,13 +120,19 @@ struct GemvArgs {
     const __half *bias;
     __half *Y;
     int32_t *C32;               // debug: raw int32 output instead of Y
-    int32_t *acc;               // split-K partials [N][16]
-    uint32_t *cnt;              // split-K arrival counters [ceil(N/32)]
+    int32_t *acc;               // partial sums of split row groups [N][M], zero on entry
+    uint32_t *cnt;              // K segments summed per group of 8 rows [ceil(N/8)], zero on entry
+    uint32_t *status;           // workspace status word (timeouts), may be null
     int64_t M, N, K;
-    int splits;
 };
-int gemv_splits(int64_t N, int64_t K);
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s);
+
+// 2-D row-major TMA map: `inner` elements per row (contiguous), `outer` rows,
+// row pitch `pitch_bytes`; box of box_inner x box_outer; out-of-range
+// elements read as zero. False if the driver rejects it.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 

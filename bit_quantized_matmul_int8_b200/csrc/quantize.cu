@@ -11,8 +11,7 @@
 //                          staged in shared memory by bulk copies; phase A
 //                          ORs the outlier columns of every row into a
 //                          bitmap, a grid barrier, then phase B writes O, CA,
-//                          SCA, Xo from the staged rows, gathers Wo and
-//                          clears the split-K buffers of the GEMV
+//                          SCA, Xo from the staged rows and gathers Wo
 //
 // Exactness: |x| >= threshold is decided on the fp16 bit pattern against the
 // smallest fp16 pattern whose value reaches the fp32 threshold (the map from
@@ -32,6 +31,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 16;  // 16-byte loads in flight per thread in phase A
+// CB up to this size is pulled into L2 for the GEMM during the quantize pass.
+constexpr int64_t kPrefetchMaxBytes = 48ll << 20;
 
 // Code of x: rint(fp32(x * s)) with s = fp32(127 / absmax) and |x| <= absmax.
 // No clamp is needed: |x * s| <= 127 * (1 + 2^-23) before rounding, so the
@@ -362,8 +363,14 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
     const uint32_t gen = s_gen;
     uint32_t *cur = a.bitmaps + (gen & 1u) * kMaxKwords;
     uint32_t *nxt = a.bitmaps + ((gen + 1u) & 1u) * kMaxKwords;
-    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
-        nxt[i] = 0;
+    // A single CTA sees every row itself: its shared bitmap is the whole
+    // outlier set, and the global bitmaps, the barrier and the launch counter
+    // are left as they are (bitmaps[gen & 1] stays zero for the next launch).
+    const bool alone = gridDim.x == 1;
+    if (!alone)
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords;
+             i += (int64_t)gridDim.x * kThreads)
+            nxt[i] = 0;
 
     // Phase A: O = { h : some |X[i,h]| >= threshold } over every row.
     for (int rd = 0; rd < rounds; ++rd) {
@@ -396,13 +403,27 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
         }
     }
     __syncthreads();
-    for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
-        if (bits[w]) atomicOr(&cur[w], bits[w]);
-    if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
+    // The prefill GEMM behind this pass streams CB; while this grid waits at
+    // its barrier and quantizes, HBM is mostly idle, so start pulling CB into
+    // L2 now (each CTA a slice; only when CB fits L2 comfortably).
+    if (a.Wo && a.CB && a.N * a.K <= kPrefetchMaxBytes && threadIdx.x < 32) {
+        const int64_t bytes = a.N * a.K;  // a multiple of 128: N % 8 == 0, K % 16 == 0
+        const int64_t slice = round_up(ceil_div(bytes, gridDim.x), 4096);
+        const int64_t b0 = (int64_t)blockIdx.x * slice, b1 = min(bytes, b0 + slice);
+        for (int64_t off = b0 + (int64_t)threadIdx.x * 4096; off < b1; off += 32 * 4096) {
+            const uint32_t n = (uint32_t)(b1 - off < 4096 ? b1 - off : 4096);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.CB + off), "r"(n) : "memory");
+        }
+    }
+    if (!alone) {
+        for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
+            if (bits[w]) atomicOr(&cur[w], bits[w]);
+        if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
+    }
 
     // Phase B: codes, scales, outlier activations; outlier-weight gather.
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
-        uint32_t v = __ldcg(&cur[w]);
+        uint32_t v = alone ? bits[w] : __ldcg(&cur[w]);
         if (w == kwords - 1 && (a.K & 31)) v &= (1u << (a.K & 31)) - 1u;
         bits[w] = v;
     }
@@ -518,11 +539,12 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
                 gather_store(t0, j0);
             }
     }
+    // Decode path: zero the GEMV's partial sums and k-block counters.
     const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x, nth = (int64_t)gridDim.x * kThreads;
     if (a.acc)
-        for (int64_t i = tid; i < a.acc_words; i += nth) a.acc[i] = 0;
+        for (int64_t i = tid; i < a.acc_words / 4; i += nth) reinterpret_cast<int4 *>(a.acc)[i] = make_int4(0, 0, 0, 0);
     if (a.cnt)
-        for (int64_t i = tid; i < a.cnt_words; i += nth) a.cnt[i] = 0;
+        for (int64_t i = tid; i < a.cnt_words / 4; i += nth) reinterpret_cast<uint4 *>(a.cnt)[i] = make_uint4(0, 0, 0, 0);
 }
 
 }  // namespace
@@ -554,6 +576,10 @@ namespace {
 
 // Largest dynamic shared memory a CTA may ask for while two still fit on an SM.
 constexpr int kQuantDynMax = 113 * 1024 - 512;
+// Batches up to this many elements (and no outlier-weight gather to spread)
+// are quantized by a single CTA.
+constexpr int64_t kAloneElems = 64 * 1024;
+constexpr int64_t kAloneClearWords = 64 * 1024;  // and at most this many decode sums to zero
 
 struct QuantOcc {
     std::mutex mu;
@@ -603,7 +629,11 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     if (r_max > 0) {
         if (cudaError_t e = quant_resident((int)(bits_bytes + r_max * row_bytes), &resident)) return e;
         if (resident <= 0) return cudaErrorInvalidConfiguration;
-        if (a.M <= r_max * resident) {
+        if (a.M <= r_max && a.M * a.K <= kAloneElems && !a.Wo && a.acc_words <= kAloneClearWords) {
+            // A small batch: one CTA, no grid-wide step at all.
+            R = (int)a.M;
+            grid = 1;
+        } else if (a.M <= r_max * resident) {
             // One round: spread the rows over every resident CTA.
             R = (int)ceil_div(a.M, resident);
             grid = (int)ceil_div(a.M, R);
@@ -618,9 +648,10 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
         if (resident <= 0) return cudaErrorInvalidConfiguration;
         grid = (int)std::min<int64_t>(resident, std::max<int64_t>(1, ceil_div(a.M, kWarps)));
     }
-    // The outlier-weight gather and the split-K clears run over all N output
-    // channels: give them enough CTAs even when there are few rows.
-    if (a.Wo || a.acc) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.N, 32)));
+    // The outlier-weight gather runs over all N output channels: give it
+    // enough CTAs even when there are few rows.
+    if (a.Wo) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.N, 32)));
+    if (a.acc) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.acc_words, kAloneClearWords)));
     if (R == 0) rounds = (int)ceil_div(a.M, (int64_t)kWarps * grid);  // kWarps rows per CTA and round
     // The grid barrier needs every CTA resident at once: a cooperative launch.
     cudaLaunchConfig_t cfg = {};

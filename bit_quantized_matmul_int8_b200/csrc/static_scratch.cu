@@ -45,8 +45,9 @@ int scratch_on_current_device(void **ptr) {
     std::call_once(g_setup_once[dev], [dev] {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-        // Start from a clean header and column bitmaps; synchronous, once.
-        if (e == cudaSuccess) e = cudaMemset(p, 0, int8lt::kWsInitBytes);
+        // Start from a zeroed scratch (as int8lt_workspace_init leaves a
+        // workspace); synchronous, once.
+        if (e == cudaSuccess) e = cudaMemset(p, 0, kStaticScratchBytes);
         g_setup_err[dev] = e;
         g_scratch_ptr[dev] = (e == cudaSuccess) ? p : nullptr;
     });
