@@ -97,7 +97,10 @@ def test_quantize_empty_batch():
 
 GEMM_SHAPES = [(128, 256, 128), (300, 520, 400), (129, 264, 4112), (1000, 776, 2048),
                (17, 8, 16), (1, 64, 64), (4, 1000, 512), (16, 4096, 1024), (3, 40, 48),
-               (4, 38400, 256), (16, 8, 4096)]
+               (4, 38400, 256), (16, 8, 4096),
+               # decode shapes whose row blocks are split between CTAs, with a
+               # short last K segment and a partial last row block
+               (5, 20000, 3008), (16, 9992, 2064)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -173,6 +176,7 @@ FCASES = [
     wl.random_case(56, 16, 4096, 1024, n_outliers=6, frac=1.0, has_bias=False),
     wl.random_case(57, 600, 2048, 1024, n_outliers=70, frac=0.2),  # > 64 outliers
     wl.random_case(58, 200, 384, 136, n_outliers=0),
+    wl.random_case(63, 7, 3008, 20000, n_outliers=5, frac=1.0),   # decode, split row blocks
 ]
 
 
