@@ -74,6 +74,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                         _P, _P, _I64, _P, _P]
     lib.oracle_outlier_weights.restype = None
     lib.oracle_outlier_weights.argtypes = [_P, _P, _P, _I64, _I64, _P, _I64, _P]
+    lib.oracle_zp_quantize_rows.restype = None
+    lib.oracle_zp_quantize_rows.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]
+    lib.oracle_zp_forward_rows.restype = None
+    lib.oracle_zp_forward_rows.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _P]
     return lib
 
 
@@ -197,3 +201,35 @@ def outlier_weights(W_outlier, CB, SCB, idx, lib=None) -> np.ndarray:
     lib.oracle_outlier_weights(_ptr(_h(W_outlier)), _ptr(CB), _ptr(SCB), N, K, _ptr(idx),
                                len(idx), _ptr(Wo))
     return Wo[:, : len(idx)].view(np.float16)
+
+
+def zp_quantize_rows(X, lib=None):
+    """Zeropoint quantization of each row: -> (codes int8 [R,K], nd fp32 [R], zp int32 [R], sum int32 [R])."""
+    lib = lib or load()
+    x = _h(X)
+    R, K = x.shape
+    Q = np.zeros((R, K), dtype=np.int8)
+    ND = np.zeros(R, dtype=np.float32)
+    ZP = np.zeros(R, dtype=np.int32)
+    SUM = np.zeros(R, dtype=np.int32)
+    lib.oracle_zp_quantize_rows(_ptr(x), R, K, _ptr(Q), _ptr(ND), _ptr(ZP), _ptr(SUM))
+    return Q, ND, ZP, SUM
+
+
+def zp_forward(X, CB, NDB, ZPB, SUMB, bias, rows=None, lib=None) -> np.ndarray:
+    """Zeropoint forward (no outlier split) -> Y64 fp64 [r, N] for rows ``rows`` (default all)."""
+    lib = lib or load()
+    x = _h(X)
+    M, K = x.shape
+    CB = np.ascontiguousarray(CB, dtype=np.int8)
+    N = CB.shape[0]
+    NDB = np.ascontiguousarray(NDB, dtype=np.float32)
+    ZPB = np.ascontiguousarray(ZPB, dtype=np.int32)
+    SUMB = np.ascontiguousarray(SUMB, dtype=np.int32)
+    if rows is None:
+        rows = np.arange(M, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    Y64 = np.zeros((len(rows), N), dtype=np.float64)
+    lib.oracle_zp_forward_rows(_ptr(x), M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZPB), _ptr(SUMB), _ptr(_h(bias)),
+                               _ptr(rows), len(rows), _ptr(Y64))
+    return Y64

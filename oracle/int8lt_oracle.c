@@ -278,3 +278,78 @@ void oracle_outlier_weights(const uint16_t *W_outlier, const int8_t *CB, const f
             Wo[j * n_out + t] =
                 oracle_double_to_half(outlier_weight(W_outlier, CB, SCB, K, j, idx[t]));
 }
+
+/* ------------------------------------ zeropoint (asymmetric) quantization -- */
+
+/* [P4 "8-bit Data Types and Quantization", zeropoint quantization] applied to
+ * one vector. The normalized dynamic range nd = 2*127 / (max - min) scales the
+ * vector; the zeropoint zp shifts it so that it spans [-127, 127]. The page's
+ * zp formula is garbled ("X * min X"); the reading taken: zp = rint(nd * min)
+ * + 127 and X_i8 = clamp(rint(nd * X) - zp, -127, 127), so that
+ * X ~= (X_i8 + zp) / nd, which is the form the page's product
+ * (A_i8 + zp_a)(B_i8 + zp_b) uses. fp32 steps as for absmax: nd is the fp32
+ * quotient of 254 by the fp32 difference max - min; products are fp32; rint
+ * rounds ties to even. A constant vector (max == min) takes nd = 1.
+ * Returns nd; *zp gets the zeropoint and *sum the sum of the codes. */
+static float zp_quantize_vector(const uint16_t *x, int64_t n, int8_t *q, int32_t *zp, int32_t *sum)
+{
+    float mn = INFINITY, mx = -INFINITY;
+    for (int64_t h = 0; h < n; ++h) {
+        float v = h2f(x[h]);
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+    }
+    if (n == 0) mn = mx = 0.0f;
+    float range = mx - mn;
+    float nd = range > 0.0f ? 254.0f / range : 1.0f;
+    float zmin = nearbyintf(mn * nd);   /* |nd * min| <= 254 * 2^10: exact in fp32 and int32 */
+    int32_t z = (int32_t)zmin + 127;
+    int64_t s = 0;
+    for (int64_t h = 0; h < n; ++h) {
+        int64_t c = (int64_t)nearbyintf(h2f(x[h]) * nd) - z;
+        if (c > 127) c = 127;
+        if (c < -127) c = -127;
+        q[h] = (int8_t)c;
+        s += c;
+    }
+    *zp = z;
+    *sum = (int32_t)s;
+    return nd;
+}
+
+/* Zeropoint quantization of every row of an fp16 matrix [R, K] (the tokens
+ * of X, or the output channels of W): codes, nd, zp and the code sums. */
+void oracle_zp_quantize_rows(const uint16_t *X, int64_t R, int64_t K, int8_t *Q, float *ND,
+                             int32_t *ZP, int32_t *SUM)
+{
+    for (int64_t i = 0; i < R; ++i) ND[i] = zp_quantize_vector(X + i * K, K, Q + i * K, ZP + i, SUM + i);
+}
+
+/* Forward with zeropoint quantization on both sides, no outlier split, for
+ * selected rows of X:
+ *   C_ij = (A_i + zp_a_i) . (B_j + zp_b_j)                         [P4]
+ *        = A_i . B_j + zp_b_j * sum(A_i) + zp_a_i * sum(B_j) + K zp_a_i zp_b_j
+ * (the page's unrolled form, in int64: the first term is the int8 GEMM, the
+ * other three are the corrections), Y_ij = C_ij / (nd_a_i nd_b_j) + bias_j
+ * in fp64. CB, NDB, ZPB, SUMB come from oracle_zp_quantize_rows on W. */
+void oracle_zp_forward_rows(const uint16_t *X, int64_t M, int64_t N, int64_t K,
+                            const int8_t *CB, const float *NDB, const int32_t *ZPB, const int32_t *SUMB,
+                            const uint16_t *bias, const int64_t *rows, int64_t nrows, double *Y64)
+{
+    int8_t *ca = (int8_t *)malloc((size_t)(K > 0 ? K : 1));
+    (void)M;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int32_t za, sa;
+        float nda = zp_quantize_vector(X + rows[r] * K, K, ca, &za, &sa);
+        for (int64_t j = 0; j < N; ++j) {
+            int64_t dot = 0;
+            const int8_t *b = CB + j * K;
+            for (int64_t k = 0; k < K; ++k) dot += (int64_t)ca[k] * (int64_t)b[k];
+            int64_t c = dot + (int64_t)ZPB[j] * sa + (int64_t)za * SUMB[j] + K * (int64_t)za * ZPB[j];
+            double y = (double)c / ((double)nda * (double)NDB[j]);
+            if (bias) y += oracle_half_to_double(bias[j]);
+            Y64[r * N + j] = y;
+        }
+    }
+    free(ca);
+}

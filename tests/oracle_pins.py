@@ -15,7 +15,12 @@ disagrees with:
 * the decomposition equation's two special cases (LLM.int8() summary,
   "Mixed-precision Decomposition"): every column an outlier gives the fp64
   matmul X W^T + bias exactly (up to fp64 rounding); and
-* a brute-force fp64 X W^T within the analytic quantization error bound.
+* a brute-force fp64 X W^T within the analytic quantization error bound;
+* for zeropoint quantization (LLM.int8() summary, "8-bit Data Types and
+  Quantization"): the row minimum maps to -127 and the maximum to 127, each
+  element is rebuilt within half a step, the unrolled product equals the
+  direct product of the shifted codes, and the forward stays within the
+  quantization error bound.
 """
 from __future__ import annotations
 
@@ -275,8 +280,85 @@ def pin_forward_within_bound(lib):
             assert np.array_equal(Y16, Y64.astype(np.float16))
 
 
+def _zp_rows(seed):
+    """Rows for the zeropoint pins: symmetric, one-sided (ReLU-like), shifted
+    far from zero, constant and all-zero rows."""
+    rng = np.random.default_rng(seed)
+    X = (rng.standard_normal((12, 61)) * rng.uniform(0.05, 4, (12, 1))).astype(np.float16)
+    X[1] = np.abs(X[1])                                    # ReLU output: one-sided
+    X[2] = (rng.uniform(100.0, 101.0, 61)).astype(np.float16)   # far from zero
+    X[3] = np.float16(2.5)                                 # constant row
+    X[4] = 0.0                                             # all-zero row
+    return X
+
+
+def pin_zp_invariants(lib):
+    """[P4 zeropoint quantization]: nd = 2*127 / (max - min) maps the row onto
+    [-127, 127]: the minimum lands on -127, the maximum on 127 (or 126 when
+    fp32 rounding of nd lands just short), and every element is rebuilt as
+    (q + zp) / nd within half a step 0.5 / nd."""
+    X = _zp_rows(3)
+    Q, ND, ZP, SUM = oracle.zp_quantize_rows(X, lib=lib)
+    Xf = X.astype(np.float64)
+    assert np.abs(Q.astype(np.int32)).max() <= 127
+    assert np.array_equal(SUM, Q.astype(np.int64).sum(axis=1))
+    for i in range(X.shape[0]):
+        mn, mx = Xf[i].min(), Xf[i].max()
+        if mx == mn:                                       # constant row
+            assert ND[i] == 1.0 and (Q[i] == -127).all()
+            assert int(Q[i, 0]) + int(ZP[i]) == int(np.rint(mn))
+            continue
+        assert abs(float(ND[i]) * (mx - mn) - 254.0) < 254.0 * 1e-6
+        assert int(Q[i, int(np.argmin(Xf[i]))]) == -127
+        assert int(Q[i, int(np.argmax(Xf[i]))]) in (126, 127)
+        rebuilt = (Q[i].astype(np.float64) + float(ZP[i])) / float(ND[i])
+        assert (np.abs(Xf[i] - rebuilt) <= 0.5 / float(ND[i]) * (1 + 1e-5)).all(), i
+    # the one-sided row uses codes on both sides of zero, unlike absmax
+    assert Q[1].min() == -127 and Q[1].max() >= 126
+    CA, _, _ = oracle.quantize_rows(X[1:2], math.inf, lib=lib)
+    assert CA.min() >= 0
+
+
+def pin_zp_unrolled_product(lib):
+    """[P4]: the unrolled form A.B + zp_b sum(A) + zp_a sum(B) + K zp_a zp_b
+    equals the direct product (A + zp_a).(B + zp_b) of the shifted codes."""
+    rng = np.random.default_rng(4)
+    X = (rng.standard_normal((7, 45)) + 0.7).astype(np.float16)
+    W = (rng.standard_normal((9, 45)) * 0.05 - 0.01).astype(np.float16)
+    b = (rng.standard_normal(9) * 0.1).astype(np.float16)
+    QA, NDA, ZA, _ = oracle.zp_quantize_rows(X, lib=lib)
+    QB, NDB, ZB, SB = oracle.zp_quantize_rows(W, lib=lib)
+    Y = oracle.zp_forward(X, QB, NDB, ZB, SB, b, lib=lib)
+    A = QA.astype(np.int64) + ZA.astype(np.int64)[:, None]
+    B = QB.astype(np.int64) + ZB.astype(np.int64)[:, None]
+    C = A @ B.T
+    want = C.astype(np.float64) / (NDA.astype(np.float64)[:, None] * NDB.astype(np.float64)[None, :])
+    want += b.astype(np.float64)[None, :]
+    assert np.array_equal(Y, want)
+
+
+def pin_zp_forward_within_bound(lib):
+    """The zeropoint forward against the fp64 X W^T + bias, within the
+    quantization error: per product |x w - x' w'| <= 0.5/nd_a |w| + |x'| 0.5/nd_b."""
+    rng = np.random.default_rng(5)
+    X = np.abs(rng.standard_normal((6, 80))).astype(np.float16)        # one-sided
+    W = (rng.standard_normal((11, 80)) * 0.05).astype(np.float16)
+    b = (rng.standard_normal(11) * 0.1).astype(np.float16)
+    QA, NDA, ZA, _ = oracle.zp_quantize_rows(X, lib=lib)
+    QB, NDB, ZB, SB = oracle.zp_quantize_rows(W, lib=lib)
+    Y = oracle.zp_forward(X, QB, NDB, ZB, SB, b, lib=lib)
+    Xf, Wf = X.astype(np.float64), W.astype(np.float64)
+    ref = Xf @ Wf.T + b.astype(np.float64)
+    ea = 0.5 / NDA.astype(np.float64)
+    eb = 0.5 / NDB.astype(np.float64)
+    bound = ea[:, None] * np.abs(Wf).sum(axis=1)[None, :] + \
+        (np.abs(Xf).sum(axis=1) + ea * X.shape[1])[:, None] * eb[None, :]
+    assert (np.abs(Y - ref) <= bound * (1 + 1e-6) + 1e-12).all()
+
+
 PINS = [pin_half_decode, pin_half_encode, pin_worked_example, pin_absmax_invariants,
         pin_weight_recovery, pin_outlier_bruteforce, pin_outlier_boundary,
         pin_planted_outliers, pin_row_scale_excludes_outliers, pin_round_ties_to_even, pin_gemm_exact,
         pin_gemm_overflow, pin_all_columns_outlier, pin_all_columns_outlier_int8_weights,
-        pin_outlier_weight_gather, pin_forward_within_bound]
+        pin_outlier_weight_gather, pin_forward_within_bound, pin_zp_invariants, pin_zp_unrolled_product,
+        pin_zp_forward_within_bound]
