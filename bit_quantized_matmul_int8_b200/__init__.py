@@ -6,7 +6,8 @@ The compute lives in ``libint8lt.so`` (CUDA, built in-tree by ``build.py``);
 from __future__ import annotations
 
 __all__ = ["Int8Linear", "int8lt_prepare_weight", "int8lt_quantize_rows", "int8lt_forward",
-           "int8lt_workspace_size", "workspace"]
+           "int8lt_workspace_size", "workspace", "int8lt_quantize_rows_zp",
+           "int8lt_prepare_weight_zp", "int8lt_forward_zp"]
 
 
 def __getattr__(name):  # import torch and the library only when used

@@ -28,6 +28,7 @@ EXPORTS = [
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
     "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
+    "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
 ]
 
 
@@ -58,6 +59,9 @@ _SIGS = {
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
     "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
     "int8lt_set_gemm_split": (ctypes.c_int, [ctypes.c_int]),
+    "int8lt_quantize_rows_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "int8lt_prepare_weight_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "int8lt_forward_zp": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -251,6 +255,50 @@ def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, ws: torch.Tensor |
 def int8lt_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
     _check("int8lt_debug_wait_timeout",
            lib().int8lt_debug_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
+
+
+def int8lt_quantize_rows_zp(X: torch.Tensor, stream=None, _fn: str = "int8lt_quantize_rows_zp"):
+    """Zeropoint quantization of each row of X fp16 [R,K] -> (Q int8 [R,K], ND fp32 [R],
+    ZP int32 [R], SUM int32 [R])."""
+    _dev(X, torch.float16, "X")
+    R, K = X.shape
+    dev = X.device
+    Q = torch.empty((R, K), dtype=torch.int8, device=dev)
+    ND = torch.empty(R, dtype=torch.float32, device=dev)
+    ZP = torch.empty(R, dtype=torch.int32, device=dev)
+    SUM = torch.empty(R, dtype=torch.int32, device=dev)
+    _check(_fn, getattr(lib(), _fn)(_ptr(X), R, K, _ptr(Q), _ptr(ND), _ptr(ZP), _ptr(SUM),
+                                    _stream(stream)))
+    return Q, ND, ZP, SUM
+
+
+def int8lt_prepare_weight_zp(W: torch.Tensor, stream=None):
+    """W fp16 [N,K] -> (CB int8 [N,K], NDB fp32 [N], ZB int32 [N], SB int32 [N])."""
+    return int8lt_quantize_rows_zp(W, stream, "int8lt_prepare_weight_zp")
+
+
+def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: torch.Tensor,
+                      SB: torch.Tensor, bias: torch.Tensor | None = None,
+                      Y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """Y fp16 [M,N]: zeropoint-quantized X times the zeropoint-quantized weight, plus bias."""
+    _dev(X, torch.float16, "X")
+    _dev(CB, torch.int8, "CB")
+    _dev(NDB, torch.float32, "NDB")
+    _dev(ZB, torch.int32, "ZB")
+    _dev(SB, torch.int32, "SB")
+    if bias is not None:
+        _dev(bias, torch.float16, "bias")
+    M, K = X.shape
+    N = CB.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    if ws is None:
+        ws = workspace(M, N, K, X.device)
+    _check("int8lt_forward_zp",
+           lib().int8lt_forward_zp(_ptr(X), M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
+                                   _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
 
 
 SPLIT_AUTO, SPLIT_ALWAYS, SPLIT_NEVER = 0, 1, 2

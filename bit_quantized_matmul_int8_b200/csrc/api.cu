@@ -23,6 +23,7 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K) {
     L.sca = off;   off += align_up((size_t)M * 4);
     L.ca = off;    off += align_up((size_t)M * K);
     L.xo = off;    off += align_up((size_t)M * L.kcap * 2);
+    L.zpa = off;   off += align_up((size_t)M * 8);
     if (M > kDecodeMaxM) {
         L.wo = off; off += align_up((size_t)N * L.kcap * 2);
         L.sk = off; off += align_up((size_t)kSkMaxPairs * 2 * kSkPartialBytes);
@@ -275,6 +276,67 @@ int int8lt_forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, con
     int st = check_forward_args(nullptr, M, N, K, CB, SCB, W_outlier, 0.f, bias, Y, false, true, ws, ws_bytes);
     if (st) return st < 0 ? INT8LT_OK : st;
     return forward_matmul(M, N, K, CB, SCB, W_outlier, bias, Y, ws, static_cast<cudaStream_t>(stream));
+}
+
+int int8lt_quantize_rows_zp(const void *X, int64_t R, int64_t K, int8_t *Q, float *ND, int32_t *ZP,
+                            int32_t *SUM, void *stream) {
+    if (!shape_ok(R, 8, K)) return INT8LT_ERR_SHAPE;
+    if (R == 0) return INT8LT_OK;
+    if (!X || !Q || !ND || !ZP || !SUM) return INT8LT_ERR_NULL;
+    if (!aligned(X, 16) || !aligned(Q, 16) || !aligned(ND, 4) || !aligned(ZP, 4) || !aligned(SUM, 4))
+        return INT8LT_ERR_ALIGN;
+    if (int st = check_device()) return st;
+    ZpQuantArgs z{};
+    z.X = static_cast<const __half *>(X); z.R = R; z.K = K;
+    z.Q = Q; z.ND = ND; z.ZP = ZP; z.SUM = SUM;
+    return from_cuda(launch_zp_quantize(z, static_cast<cudaStream_t>(stream)));
+}
+
+int int8lt_prepare_weight_zp(const void *W, int64_t N, int64_t K, int8_t *CB, float *NDB, int32_t *ZB,
+                             int32_t *SB, void *stream) {
+    if (!shape_ok(8, N, K)) return INT8LT_ERR_SHAPE;
+    return int8lt_quantize_rows_zp(W, N, K, CB, NDB, ZB, SB, stream);
+}
+
+int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *NDB,
+                      const int32_t *ZB, const int32_t *SB, const void *bias, void *Y, void *ws, size_t ws_bytes,
+                      void *stream) {
+    int st = check_forward_args(X, M, N, K, CB, NDB, nullptr, 0.f, bias, Y, true, true, ws, ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
+    if (!ZB || !SB) return INT8LT_ERR_NULL;
+    if (!aligned(ZB, 4) || !aligned(SB, 4)) return INT8LT_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(M, N, K);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    int8_t *CA = at<int8_t>(ws, L.ca);
+    float *NDA = at<float>(ws, L.sca);
+    int32_t *ZA = at<int32_t>(ws, L.zpa), *SA = ZA + M;
+    const bool decode = M <= kDecodeMaxM;
+    ZpQuantArgs z{};
+    z.X = static_cast<const __half *>(X); z.R = M; z.K = K;
+    z.Q = CA; z.ND = NDA; z.ZP = ZA; z.SUM = SA;
+    if (decode) {  // the GEMV's partial sums and counters start at zero
+        z.acc = at<int32_t>(ws, L.acc); z.acc_words = round_up(N * M, 4);
+        z.cnt = at<uint32_t>(ws, L.cnt); z.cnt_words = round_up(ceil_div(N, 8), 4);
+    }
+    if ((st = from_cuda(launch_zp_quantize(z, s)))) return st;
+    if (decode) {
+        GemvArgs g{};
+        g.CA = CA; g.CB = CB; g.SCA = NDA; g.SCB = NDB;
+        g.ZA = ZA; g.SA = SA; g.ZB = ZB; g.SB = SB;
+        g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
+        g.acc = at<int32_t>(ws, L.acc); g.cnt = at<uint32_t>(ws, L.cnt); g.status = &hdr->status;
+        g.M = M; g.N = N; g.K = K;
+        return from_cuda(launch_gemv(g, s));
+    }
+    GemmArgs g{};
+    g.CA = CA; g.CB = CB; g.SCA = NDA; g.SCB = NDB;
+    g.ZA = ZA; g.SA = SA; g.ZB = ZB; g.SB = SB;
+    g.bias = static_cast<const __half *>(bias); g.Y = static_cast<__half *>(Y);
+    g.M = M; g.N = N; g.K = K; g.status = &hdr->status;
+    g.sk_partial = at<int32_t>(ws, L.sk);
+    g.sk_flags = at<uint32_t>(ws, kWsSkFlagOffset);
+    return from_cuda(launch_gemm_tc(g, s));
 }
 
 int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K, int32_t *C,

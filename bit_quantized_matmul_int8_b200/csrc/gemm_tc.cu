@@ -157,7 +157,9 @@ constexpr size_t kOffStage = kOffOut + 2 * (size_t)kOStage;      // [kEpiWarps][
 constexpr size_t kOffCtrl = kOffStage + (size_t)kEpiWarps * kBoxes * kStoreBufBytes;
 constexpr size_t kOffScb = kOffCtrl + 256;
 constexpr size_t kOffBias = kOffScb + BN * 4;
-constexpr size_t kSmemUsed = kOffBias + BN * 4;
+constexpr size_t kOffZb = kOffBias + BN * 4;   // zeropoint mode: zp_b of the tile's columns
+constexpr size_t kOffSb = kOffZb + BN * 4;     // zeropoint mode: code sums of the tile's columns
+constexpr size_t kSmemUsed = kOffSb + BN * 4;
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kSmemUsed;
 static_assert(sizeof(Ctrl) <= 256, "control block");
 static_assert(kOffOut % 1024 == 0 && kOStage % 1024 == 0, "swizzle atoms need aligned slots");
@@ -241,6 +243,33 @@ __device__ __forceinline__ void dequant32(uint32_t (&acc)[32], float rs, const f
     }
 }
 
+// Zeropoint mode: acc (int32 sums A.B of 32 columns, plus the tail's partial
+// sums if any) -> fp32 (C + zb_j * ta + za * sb_j) * inv_a * inv_b_j + bias_j,
+// the unrolled (A + zp_a)(B + zp_b) product of "8-bit Data Types and
+// Quantization" (zeropoint quantization) with ta = sa + K * za. The
+// correction is added in int64 (exact), then converted to fp32 once.
+__device__ __forceinline__ void dequant32_zp(uint32_t (&acc)[32], float inv_a, int64_t ta, int32_t za,
+                                             const float *s_invb, const float *s_bias, const int32_t *s_zb,
+                                             const int32_t *s_sb, const int4 *part, int cc) {
+    add_partial(acc, part, cc);
+    const float4 *ib4 = reinterpret_cast<const float4 *>(s_invb);
+    const float4 *bi4 = reinterpret_cast<const float4 *>(s_bias);
+    const int4 *zb4 = reinterpret_cast<const int4 *>(s_zb);
+    const int4 *sb4 = reinterpret_cast<const int4 *>(s_sb);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const float4 ib = ib4[v], bi = bi4[v];
+        const int4 zb = zb4[v], sb = sb4[v];
+        const float ibv[4] = {ib.x, ib.y, ib.z, ib.w}, biv[4] = {bi.x, bi.y, bi.z, bi.w};
+        const int32_t zbv[4] = {zb.x, zb.y, zb.z, zb.w}, sbv[4] = {sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t c = (int64_t)(int32_t)acc[4 * v + e] + (int64_t)zbv[e] * ta + (int64_t)za * sbv[e];
+            acc[4 * v + e] = __float_as_uint(__fmaf_rn(__fmul_rn(__ll2float_rn(c), inv_a), ibv[e], biv[e]));
+        }
+    }
+}
+
 // fp32 (bit patterns) -> fp16, staged in the warp's next 32 x 32 box in shared
 // memory (64-byte swizzle: 16-byte chunk i of row r sits at chunk
 // i ^ ((r >> 1) & 3), which keeps the four stores of each row conflict-free)
@@ -272,6 +301,7 @@ __device__ __forceinline__ void store32(const uint32_t (&y)[32], uint8_t *s_stag
     sbuf = kBoxes == 2 ? sbuf ^ 1 : 0;
 }
 
+template <bool kZp>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmXo, const __grid_constant__ CUtensorMap tmWo,
@@ -286,6 +316,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem + kOffCtrl);
     float *s_scb = reinterpret_cast<float *>(smem + kOffScb);
     float *s_bias = reinterpret_cast<float *>(smem + kOffBias);
+    int32_t *s_zb = reinterpret_cast<int32_t *>(smem + kOffZb);
+    int32_t *s_sb = reinterpret_cast<int32_t *>(smem + kOffSb);
     uint8_t *s_stage = smem + kOffStage;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -332,7 +364,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // reads what the quantize pass wrote (launched with programmatic stream
     // serialization, the prologue overlaps the end of that pass).
     grid_dep_wait();
-    const int n_out = (a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
+    const int n_out = (!kZp && a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
     const int n_okb = (n_out + kOkb - 1) / kOkb;       // outlier k-blocks per tile
     const int n_mma_o = (n_out + 15) >> 4;             // fp16 MMAs of K = 16 per tile
     const uint32_t tmem = ctrl->tmem_base;
@@ -547,11 +579,25 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // and this thread's row scale while the MMAs are still running.
             const int64_t col = n0 + et;
             const bool col_ok = !a.C32 && et < BN && col < a.N;
-            const float scb_v = col_ok ? a.SCB[col] : 0.f;
+            // (Zeropoint mode: 1 / nd_b, zp_b and the code sums per column;
+            // 1 / nd_a, zp_a and sa + K zp_a for the row.)
+            const float scb_v = col_ok ? (kZp ? 1.0f / a.SCB[col] : a.SCB[col]) : 0.f;
             const float bias_v = (col_ok && a.bias) ? __half2float(a.bias[col]) : 0.f;
             const int64_t row = m0 + q * 32 + lane;
             const bool row_ok = row < a.M;
-            const float sca_v = (row_ok && a.SCA) ? a.SCA[row] : 0.f;
+            const float sca_v = (row_ok && a.SCA) ? (kZp ? 1.0f / a.SCA[row] : a.SCA[row]) : 0.f;
+            int32_t zb_v = 0, sb_v = 0, za_v = 0;
+            int64_t ta_v = 0;
+            if constexpr (kZp) {
+                if (col_ok) {
+                    zb_v = a.ZB[col];
+                    sb_v = a.SB[col];
+                }
+                if (row_ok) {
+                    za_v = a.ZA[row];
+                    ta_v = (int64_t)a.SA[row] + a.K * (int64_t)za_v;
+                }
+            }
             // Wait for the accumulator, then decide together whether to go
             // on: every epilogue warp votes before the barrier and reads the
             // same slot after it, so all of them leave the loop together.
@@ -569,6 +615,10 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (!a.C32 && et < BN) {
                 s_scb[et] = scb_v;
                 s_bias[et] = bias_v;
+                if constexpr (kZp) {
+                    s_zb[et] = zb_v;
+                    s_sb[et] = sb_v;
+                }
             }
             epi_sync();
             tc_fence_after();
@@ -669,7 +719,11 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         if (lane == 0) arrive_leader(ctrl, &ctrl->acc_empty[buf], rank);
                     }
                     if (n0 + hcol * kEpiCols + cc >= a.N) continue;  // whole chunk past the last column
-                    dequant32(acc, rs, s_scb + hcol * kEpiCols + cc, s_bias + hcol * kEpiCols + cc, part, cc);
+                    const int sc = hcol * kEpiCols + cc;
+                    if constexpr (kZp)
+                        dequant32_zp(acc, sca_v, ta_v, za_v, s_scb + sc, s_bias + sc, s_zb + sc, s_sb + sc, part, cc);
+                    else
+                        dequant32(acc, rs, s_scb + sc, s_bias + sc, part, cc);
                     store32(acc, s_stage, ew, sbuf, lane, &tmY, (int32_t)(n0 + hcol * kEpiCols + cc),
                             (int32_t)(m0 + q * 32));
                 }
@@ -774,13 +828,17 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     std::call_once(attr_once[dev & 63], [&] {
-        attr_err = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        attr_err = cudaFuncSetAttribute(gemm_i8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)kSmemBytes);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gemm_i8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)kSmemBytes);
         if (attr_err != cudaSuccess) return;
         // How many CTA pairs can be resident at once (a pair needs two SMs of one GPC).
         cudaLaunchConfig_t q = cfg;
         q.gridDim = dim3(2, 1, 1);
         int clusters = 0;
-        attr_err = cudaOccupancyMaxActiveClusters(&clusters, (void *)gemm_i8_kernel, &q);
+        attr_err = cudaOccupancyMaxActiveClusters(&clusters, (void *)gemm_i8_kernel<false>, &q);
         g_num_sms[dev & 63] = clusters;
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -795,7 +853,12 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     }
     cfg.gridDim = dim3(2 * (unsigned)grid_pairs, 1, 1);
     cfg.numAttrs = 2;  // and programmatic stream serialization
-    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel, mA, mB, mXo, mWo, mY, b, num_m_tiles, (int)tiles);
+    if (a.ZB) {  // zeropoint mode: no outlier term
+        if (!a.ZA || !a.SA || !a.SB || !a.SCA || !a.SCB || a.C32) return cudaErrorInvalidValue;
+        b.n_outliers = nullptr;
+        return cudaLaunchKernelEx(&cfg, gemm_i8_kernel<true>, mA, mB, mXo, mWo, mY, b, num_m_tiles, (int)tiles);
+    }
+    return cudaLaunchKernelEx(&cfg, gemm_i8_kernel<false>, mA, mB, mXo, mWo, mY, b, num_m_tiles, (int)tiles);
 }
 
 }  // namespace int8lt

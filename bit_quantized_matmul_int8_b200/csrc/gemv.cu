@@ -71,6 +71,15 @@ __device__ __forceinline__ float outlier_weight(const GemvArgs &a, int64_t j, in
 // Final value of output (token t, channel j) from its int32 sum.
 __device__ __forceinline__ void finish(const GemvArgs &a, int n_out, int64_t t, int64_t j, int32_t c,
                                        float &y) {
+    if (a.ZB) {
+        // Zeropoint mode: (A + zp_a)(B + zp_b) unrolled into the int8 sum and
+        // three exact int64 corrections ("8-bit Data Types and Quantization").
+        const int64_t za = a.ZA[t], zb = a.ZB[j];
+        const int64_t ct = (int64_t)c + zb * ((int64_t)a.SA[t] + a.K * za) + za * (int64_t)a.SB[j];
+        y = __fmul_rn(__ll2float_rn(ct), 1.0f / a.SCA[t]) * (1.0f / a.SCB[j]);
+        if (a.bias) y += __half2float(a.bias[j]);
+        return;
+    }
     y = (float)c * (a.SCA[t] * (1.0f / 16129.0f) * a.SCB[j]);
     float p = 0.f;
     for (int o = 0; o < n_out; ++o)
@@ -169,7 +178,7 @@ gemv_i8_kernel(const GemvArgs a, const int64_t row_groups, const int splits) {
             }
     }
 
-    const int n_out = a.n_outliers ? *a.n_outliers : 0;
+    const int n_out = (a.n_outliers && !a.ZB) ? *a.n_outliers : 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll

@@ -29,7 +29,9 @@ struct WsLayout {
     int64_t M, N, K;
     int64_t kwords;        // ceil(K / 32): words of one column bitmap
     int64_t kcap;          // round_up(K, 64): row pitch (elements) of Xo / Wo
-    size_t hdr, bitmaps, idx, sca, ca, xo, wo, acc, cnt, sk, total;
+    size_t hdr, bitmaps, idx, sca, ca, xo, wo, acc, cnt, sk;
+    size_t zpa;            // zeropoint forward: zp_a [M] then the code sums [M] (int32)
+    size_t total;
 };
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K);
 
@@ -87,6 +89,22 @@ struct QuantizeArgs {
 // flags of every row, a grid barrier, then codes/scales/outlier gathers.
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 
+// Zeropoint quantization of the rows of an fp16 matrix [R, K] (K % 8 == 0).
+struct ZpQuantArgs {
+    const __half *X;
+    int64_t R, K;
+    int8_t *Q;                // [R, K] codes
+    float *ND;                // [R]
+    int32_t *ZP;              // [R]
+    int32_t *SUM;             // [R]
+    // Decode path: partial-sum buffers to zero for the GEMV, or null.
+    int32_t *acc;
+    int64_t acc_words;        // a multiple of 4
+    uint32_t *cnt;
+    int64_t cnt_words;        // a multiple of 4
+};
+cudaError_t launch_zp_quantize(const ZpQuantArgs &a, cudaStream_t s);
+
 struct GemmArgs {
     const int8_t *CA;
     const int8_t *CB;
@@ -104,6 +122,9 @@ struct GemmArgs {
     // Stream-K of the last wave (both null: whole tiles only).
     int32_t *sk_partial;      // [kSkMaxPairs][2][128][256]
     uint32_t *sk_flags;       // [kSkMaxPairs][2], zero between launches
+    // Zeropoint mode (ZB non-null): SCA / SCB hold nd_a / nd_b, no outlier term.
+    const int32_t *ZA, *SA;   // [M] zeropoints and code sums of the rows of CA
+    const int32_t *ZB, *SB;   // [N] zeropoints and code sums of the rows of CB
 };
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 
@@ -124,6 +145,9 @@ struct GemvArgs {
     uint32_t *cnt;              // K segments summed per group of 8 rows [ceil(N/8)], zero on entry
     uint32_t *status;           // workspace status word (timeouts), may be null
     int64_t M, N, K;
+    // Zeropoint mode (ZB non-null): SCA / SCB hold nd_a / nd_b, no outlier term.
+    const int32_t *ZA, *SA;     // [M]
+    const int32_t *ZB, *SB;     // [N]
 };
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s);
 

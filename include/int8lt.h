@@ -193,6 +193,48 @@ int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N, int64_t K
                                   const int8_t *CB, const float *SCB, const void *W_outlier,
                                   float threshold, const void *bias, void *Y, void *stream);
 
+/* ------------------------------------------------- zeropoint quantization -- */
+
+/*
+ * Zeropoint (asymmetric) row quantization, [P] "8-bit Data Types and
+ * Quantization", zeropoint quantization: every row x of X fp16 [R, K] (a
+ * token of an activation matrix, or an output channel of W) gets
+ *   ND[i]  = fp32(254 / fp32(max x - min x))   (1 when max x == min x),
+ *   ZP[i]  = rint(fp32(ND[i] * min x)) + 127,
+ *   Q[i,h] = clamp(rint(fp32(ND[i] * X[i,h])) - ZP[i], -127, 127),
+ *   SUM[i] = sum over h of Q[i,h],
+ * rint rounding ties to even, so that X[i,h] ~= (Q[i,h] + ZP[i]) / ND[i]. The
+ * page's zeropoint formula is garbled; this is the reading whose shifted
+ * codes the page's product (A + zp_a)(B + zp_b) takes. Unlike absmax codes,
+ * the full [-127, 127] range is used by every row whatever its sign balance.
+ *   Q   : int8 [R, K] (16-byte aligned); ND fp32 [R]; ZP, SUM int32 [R].
+ * K % 16 == 0, 16 <= K <= 133144 (as for int8lt_forward). Deterministic; no
+ * workspace. int8lt_prepare_weight_zp is the same operation on W [N, K]
+ * (N % 8 == 0), written CB / NDB / ZB / SB for int8lt_forward_zp.
+ */
+int int8lt_quantize_rows_zp(const void *X, int64_t R, int64_t K, int8_t *Q, float *ND,
+                            int32_t *ZP, int32_t *SUM, void *stream);
+int int8lt_prepare_weight_zp(const void *W, int64_t N, int64_t K, int8_t *CB, float *NDB,
+                             int32_t *ZB, int32_t *SB, void *stream);
+
+/*
+ * Linear layer with zeropoint quantization on both sides and no outlier
+ * split ([P] "8-bit Data Types and Quantization": the product of two
+ * zeropoint-quantized operands, unrolled):
+ *   C[i,j] = (A_i + za_i) . (B_j + zb_j)
+ *          = A_i . B_j + zb_j SA_i + za_i SB_j + K za_i zb_j,
+ *   Y[i,j] = fp16( C[i,j] / (NDA[i] NDB[j]) + bias[j] ),
+ * where A, NDA, za, SA are the zeropoint codes of the rows of X (computed by
+ * this call into the workspace) and CB, NDB, ZB, SB come from
+ * int8lt_prepare_weight_zp. A_i . B_j runs on the int8 tensor cores (int32,
+ * exact); the corrections are added in int64 (exact) and the sum is scaled
+ * in fp32. Same dispatch, shapes, alignment and workspace
+ * (int8lt_workspace_size) as int8lt_forward; ZB and SB 4-byte aligned.
+ */
+int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K,
+                      const int8_t *CB, const float *NDB, const int32_t *ZB, const int32_t *SB,
+                      const void *bias, void *Y, void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- tests -- */
 
 /*
