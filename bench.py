@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--out", default=None, help="also append the JSON line to this file")
+    p.add_argument("--quant", choices=["absmax", "zeropoint"], default="absmax",
+                   help="absmax + outlier decomposition (LLM.int8()), or zeropoint on both sides")
     return p.parse_args()
 
 
@@ -159,35 +161,46 @@ class ClockSampler:
 
 # --------------------------------------------------------------- CPU oracle --
 
-def cpu_oracle_sample(w: wl.Workload, target_s: float, X=None, W=None):
-    """Time the oracle forward on the first r rows of the workload (r sized to target_s)."""
+def oracle_forward(w: wl.Workload, X, W, b, quant: str):
+    """The oracle's forward of the chosen quantization, as a function of the row sample."""
     import oracle
 
+    if quant == "zeropoint":
+        CB, NDB, ZB, SB = oracle.zp_quantize_rows(W)
+        return lambda rows: oracle.zp_forward(X, CB, NDB, ZB, SB, b, rows=rows)
+    CB, SCB = oracle.prepare_weight(W)
+    return lambda rows: oracle.forward(X, CB, SCB, W, w.threshold, b, rows=rows)
+
+
+def cpu_oracle_sample(w: wl.Workload, target_s: float, X=None, W=None, quant: str = "absmax"):
+    """Time the oracle forward on the first r rows of the workload (r sized to target_s)."""
     if X is None:
         X = wl.make_x(w)
     if W is None:
         W = wl.make_w(w)
     b = wl.make_bias(w)
-    CB, SCB = oracle.prepare_weight(W)       # weight conversion: offline, not timed
+    fwd = oracle_forward(w, X, W, b, quant)   # weight conversion inside: offline, not timed
     probe = min(w.M, 8)
     t0 = time.perf_counter()
-    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(probe))
+    fwd(np.arange(probe))
     per_row = (time.perf_counter() - t0) / probe          # upper bound: includes fixed costs
     rows = int(max(1, min(w.M, target_s / max(per_row, 1e-6))))
     t0 = time.perf_counter()
-    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(rows))
+    fwd(np.arange(rows))
     dt = time.perf_counter() - t0
     if dt < 0.5 * target_s and rows < w.M:
         # the probe's fixed costs made the first sample short: size it again
         rows = int(max(1, min(w.M, rows * target_s / max(dt, 1e-6))))
         t0 = time.perf_counter()
-        oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(rows))
+        fwd(np.arange(rows))
         dt = time.perf_counter() - t0
     ops = 2.0 * rows * w.N * w.K
+    what = ("outlier set over all rows, row quantize, int64-checked int8 GEMM, fp64 dequant + "
+            "outlier product" if quant == "absmax" else
+            "zeropoint row quantize, int64 int8 GEMM + zeropoint corrections, fp64 scale")
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of {w.M} rows x all {w.N} output channels (outlier set over "
-                      f"all rows, row quantize, int64-checked int8 GEMM, fp64 dequant + outlier "
-                      f"product); {dt:.2f} s on 1 host core",
+            "sample": f"first {rows} of {w.M} rows x all {w.N} output channels ({what}); "
+                      f"{dt:.2f} s on 1 host core",
             "host_cores": os.cpu_count(), "seconds": dt, "rows": rows}
 
 
@@ -195,23 +208,21 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     w = wl.WORKLOADS[args.workload]
-    import oracle
-
     X, W = wl.make_x(w), wl.make_w(w)
     b = wl.make_bias(w)
-    CB, SCB = oracle.prepare_weight(W)
+    fwd = oracle_forward(w, X, W, b, args.quant)
     t0 = time.perf_counter()
-    oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(1))
+    fwd(np.arange(1))
     t_row = time.perf_counter() - t0
     budget = 150.0 / max(1, args.steps + args.warmup)      # whole run ~ 2.5 minutes
     rows = int(max(1, min(w.M, budget / max(t_row, 1e-6))))
     for _ in range(args.warmup):
-        oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(rows))
+        fwd(np.arange(rows))
     times = []
     for s in range(args.steps):
         r0 = (s * rows) % max(1, w.M - rows + 1)
         t0 = time.perf_counter()
-        oracle.forward(X, CB, SCB, W, w.threshold, b, rows=np.arange(r0, r0 + rows))
+        fwd(np.arange(r0, r0 + rows))
         times.append(time.perf_counter() - t0)
     total = sum(times)
     ops = 2.0 * rows * w.N * w.K * args.steps
@@ -222,7 +233,7 @@ def run_reference(args, rank: int, world: int):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "n_outliers": w.n_outliers,
-                   "threshold": w.threshold, "rows_per_step": rows},
+                   "threshold": w.threshold, "rows_per_step": rows, "quant": args.quant},
         "tokens_per_s": rows * args.steps / total,
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
                          "sample": f"{rows} of {w.M} rows per step, all {w.N} output channels"},
@@ -276,8 +287,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     Xh = torch.from_numpy(X).pin_memory()
     Wd = torch.from_numpy(W).to(dev)
     bd = torch.from_numpy(b).to(dev) if b is not None else None
-    CB0, SCB = _lib.int8lt_prepare_weight(Wd)
+    zp = args.quant == "zeropoint"
+    if zp:
+        CB0, NDB, ZB, SB = _lib.int8lt_prepare_weight_zp(Wd)
+    else:
+        CB0, SCB = _lib.int8lt_prepare_weight(Wd)
     torch.cuda.synchronize()
+
+    # The forward and its two halves, on one input set.
+    def fwd(Xd, CB, Y, ws, st):
+        if zp:
+            _lib.int8lt_forward_zp(Xd, CB, NDB, ZB, SB, bd, Y, ws, st)
+        else:
+            _lib.int8lt_forward(Xd, CB, SCB, Wd, w.threshold, bd, Y, ws, st)
+
+    def fwd_quantize(Xd, CB, ws, st):
+        if zp:
+            _lib.int8lt_forward_zp_quantize(Xd, N, ws, st)
+        else:
+            _lib.int8lt_forward_quantize(Xd, CB, SCB, Wd, w.threshold, ws, st)
+
+    def fwd_matmul(CB, Y, ws, st):
+        if zp:
+            _lib.int8lt_forward_zp_matmul(M, CB, NDB, ZB, SB, bd, Y, ws, st)
+        else:
+            _lib.int8lt_forward_matmul(M, CB, SCB, Wd, bd, Y, ws, st)
 
     # Rotating input sets: X, CB, Y and workspace per set.
     ws_bytes = _lib.int8lt_workspace_size(M, N, K)
@@ -292,7 +326,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     def step(s):
         r = s % R
-        _lib.int8lt_forward(Xs[r], CBs[r], SCB, Wd, w.threshold, bd, Ys[r], WSs[r], stream)
+        fwd(Xs[r], CBs[r], Ys[r], WSs[r], stream)
 
     for s in range(max(3, args.warmup)):
         step(s)
@@ -313,9 +347,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         with torch.cuda.graph(g, stream=cap_stream):
             cs = torch.cuda.current_stream()
             evq[s].record(cs)
-            _lib.int8lt_forward_quantize(Xs[r], CBs[r], SCB, Wd, w.threshold, WSs[r], cs)
+            fwd_quantize(Xs[r], CBs[r], WSs[r], cs)
             evm[s].record(cs)
-            _lib.int8lt_forward_matmul(M, CBs[r], SCB, Wd, bd, Ys[r], WSs[r], cs)
+            fwd_matmul(CBs[r], Ys[r], WSs[r], cs)
             eve[s].record(cs)
         graphs.append(g)
     for g in graphs[: min(len(graphs), max(3, args.warmup))]:
@@ -357,7 +391,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     src = ["bit_quantized_matmul_int8_b200/csrc/gemm_tc.cu" if not decode
            else "bit_quantized_matmul_int8_b200/csrc/gemv.cu",
            "bit_quantized_matmul_int8_b200/csrc/int8lt_internal.cuh"]
-    kname = ("gemm_i8_kernel" if not decode else "gemv_i8_kernel") + "@" + w.name
+    kname = (("gemm_i8_kernel" if not decode else "gemv_i8_kernel") + ("<zp>" if zp else "")
+             + "@" + w.name)
     traffic = dram_traffic(kname, src)
     if not decode:
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -368,14 +403,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                f"(int8/bf16 nominal ratio)",
                 "algorithmic_units": f"2*M*N*K = {ops:.4g} int8 ops per launch"}
     else:
-        n_out = w.n_outliers if math.isfinite(w.threshold) else 0
-        alg_bytes = N * K + 4 * N + M * K + 4 * M + 2 * M * N + 2 * M * n_out + 2 * N * n_out
+        if zp:  # CB + NDB/ZB/SB + CA + NDA/ZA/SA + Y
+            alg_bytes = N * K + 12 * N + M * K + 12 * M + 2 * M * N
+        else:
+            n_out = w.n_outliers if math.isfinite(w.threshold) else 0
+            alg_bytes = N * K + 4 * N + M * K + 4 * M + 2 * M * N + 2 * M * n_out + 2 * N * n_out
         achieved = alg_bytes / m_avg / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": "gemv_i8_kernel", "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peaks['source']} HBM copy",
-                "algorithmic_units": f"{alg_bytes} bytes per launch (CB + SCB + CA + SCA + Y + outliers)"}
+                "algorithmic_units": f"{alg_bytes} bytes per launch (CB + SCB + CA + SCA + Y + outliers)"
+                                     if not zp else f"{alg_bytes} bytes per launch (CB + NDB/ZB/SB + CA"
+                                                    f" + NDA/ZA/SA + Y)"}
 
     # End to end through the public API: pinned X -> device, forward, Y -> pinned host.
     Yh = torch.empty((M, N), dtype=torch.float16).pin_memory()
@@ -384,7 +424,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     Yd = torch.empty_like(Ys[0])
     for _ in range(3):
         Xd.copy_(Xh, non_blocking=True)
-        _lib.int8lt_forward(Xd, CBs[0], SCB, Wd, w.threshold, bd, Yd, layer_ws, stream)
+        fwd(Xd, CBs[0], Yd, layer_ws, stream)
         Yh.copy_(Yd, non_blocking=True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -395,7 +435,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e0.record()
     for _ in range(n_e2e):
         Xd.copy_(Xh, non_blocking=True)
-        _lib.int8lt_forward(Xd, CBs[0], SCB, Wd, w.threshold, bd, Yd, layer_ws, stream)
+        fwd(Xd, CBs[0], Yd, layer_ws, stream)
         Yh.copy_(Yd, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
@@ -414,16 +454,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "threshold": w.threshold, "x": "N(0,1) fp16 + planted outlier columns",
                    "w": f"N(0,{w.sigma_w}) fp16", "l2": f"{R} rotating input sets "
                    f"({R * touched / 2**20:.0f} MiB touched per cycle) > 126 MB L2",
-                   "parallelism": f"replicas x{world}", "cuda_graphs": True},
+                   "parallelism": f"replicas x{world}", "cuda_graphs": True, "quant": args.quant},
         "tokens_per_s": tokens_per_s,
         "phases_ms": {"quantize": q_avg * 1e3, "matmul": m_avg * 1e3},
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": K_steps * 2,  # quantize_kernel + the GEMM or GEMV, per step
+        "gpu_launches": K_steps * 2,  # the quantize kernel + the GEMM or GEMV, per step
         "clocks": sampler.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W)
+        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W, args.quant)
     elif not args.no_cpu_baseline:
         line["cpu_baseline"] = None
     emit(line, args.out)

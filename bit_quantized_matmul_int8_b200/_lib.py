@@ -29,6 +29,7 @@ EXPORTS = [
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
     "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
     "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
+    "int8lt_forward_zp_quantize", "int8lt_forward_zp_matmul",
 ]
 
 
@@ -62,6 +63,8 @@ _SIGS = {
     "int8lt_quantize_rows_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "int8lt_prepare_weight_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "int8lt_forward_zp": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "int8lt_forward_zp_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "int8lt_forward_zp_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -299,6 +302,24 @@ def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: 
            lib().int8lt_forward_zp(_ptr(X), M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
                                    _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
     return Y
+
+
+def int8lt_forward_zp_quantize(X: torch.Tensor, N: int, ws: torch.Tensor, stream=None) -> None:
+    """First half of int8lt_forward_zp: zeropoint-quantize X's rows into ws."""
+    M, K = X.shape
+    _check("int8lt_forward_zp_quantize",
+           lib().int8lt_forward_zp_quantize(_ptr(X), M, N, K, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def int8lt_forward_zp_matmul(M: int, CB: torch.Tensor, NDB: torch.Tensor, ZB: torch.Tensor,
+                             SB: torch.Tensor, bias: torch.Tensor | None, Y: torch.Tensor,
+                             ws: torch.Tensor, stream=None) -> None:
+    """Second half of int8lt_forward_zp: GEMM/GEMV with the zeropoint epilogue into Y."""
+    N, K = CB.shape
+    _check("int8lt_forward_zp_matmul",
+           lib().int8lt_forward_zp_matmul(M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
+                                          _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
 
 
 SPLIT_AUTO, SPLIT_ALWAYS, SPLIT_NEVER = 0, 1, 2

@@ -113,6 +113,15 @@ int check_forward_args(const void *X, int64_t M, int64_t N, int64_t K, const int
     return check_device();
 }
 
+// The zeropoint forward's extra weight arrays (-1: empty output, nothing to check).
+int check_zp_weight_args(int64_t M, int64_t N, int64_t K, const int32_t *ZB, const int32_t *SB) {
+    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (M == 0 || N == 0) return -1;
+    if (!ZB || !SB) return INT8LT_ERR_NULL;
+    if (!aligned(ZB, 4) || !aligned(SB, 4)) return INT8LT_ERR_ALIGN;
+    return 0;
+}
+
 }  // namespace
 
 namespace int8lt {
@@ -298,29 +307,39 @@ int int8lt_prepare_weight_zp(const void *W, int64_t N, int64_t K, int8_t *CB, fl
     return int8lt_quantize_rows_zp(W, N, K, CB, NDB, ZB, SB, stream);
 }
 
-int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *NDB,
-                      const int32_t *ZB, const int32_t *SB, const void *bias, void *Y, void *ws, size_t ws_bytes,
-                      void *stream) {
-    int st = check_forward_args(X, M, N, K, CB, NDB, nullptr, 0.f, bias, Y, true, true, ws, ws_bytes);
-    if (st) return st < 0 ? INT8LT_OK : st;
-    if (!ZB || !SB) return INT8LT_ERR_NULL;
-    if (!aligned(ZB, 4) || !aligned(SB, 4)) return INT8LT_ERR_ALIGN;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+int int8lt_forward_zp_quantize(const void *X, int64_t M, int64_t N, int64_t K, void *ws, size_t ws_bytes,
+                               void *stream) {
+    if (!shape_ok(M, N, K)) return INT8LT_ERR_SHAPE;
+    if (M == 0 || N == 0) return INT8LT_OK;
+    if (!X || !ws) return INT8LT_ERR_NULL;
+    if (!aligned(X, 16) || !aligned(ws, 16)) return INT8LT_ERR_ALIGN;
     const WsLayout L = ws_layout(M, N, K);
-    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
-    int8_t *CA = at<int8_t>(ws, L.ca);
-    float *NDA = at<float>(ws, L.sca);
-    int32_t *ZA = at<int32_t>(ws, L.zpa), *SA = ZA + M;
-    const bool decode = M <= kDecodeMaxM;
+    if (ws_bytes < L.total) return INT8LT_ERR_WORKSPACE;
+    if (int st = check_device()) return st;
     ZpQuantArgs z{};
     z.X = static_cast<const __half *>(X); z.R = M; z.K = K;
-    z.Q = CA; z.ND = NDA; z.ZP = ZA; z.SUM = SA;
-    if (decode) {  // the GEMV's partial sums and counters start at zero
+    z.Q = at<int8_t>(ws, L.ca); z.ND = at<float>(ws, L.sca);
+    z.ZP = at<int32_t>(ws, L.zpa); z.SUM = z.ZP + M;
+    if (M <= kDecodeMaxM) {  // the GEMV's partial sums and counters start at zero
         z.acc = at<int32_t>(ws, L.acc); z.acc_words = round_up(N * M, 4);
         z.cnt = at<uint32_t>(ws, L.cnt); z.cnt_words = round_up(ceil_div(N, 8), 4);
     }
-    if ((st = from_cuda(launch_zp_quantize(z, s)))) return st;
-    if (decode) {
+    return from_cuda(launch_zp_quantize(z, static_cast<cudaStream_t>(stream)));
+}
+
+int int8lt_forward_zp_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *NDB,
+                             const int32_t *ZB, const int32_t *SB, const void *bias, void *Y, void *ws,
+                             size_t ws_bytes, void *stream) {
+    int st = check_zp_weight_args(M, N, K, ZB, SB);
+    if (!st) st = check_forward_args(nullptr, M, N, K, CB, NDB, nullptr, 0.f, bias, Y, false, true, ws, ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(M, N, K);
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    const int8_t *CA = at<int8_t>(ws, L.ca);
+    const float *NDA = at<float>(ws, L.sca);
+    const int32_t *ZA = at<int32_t>(ws, L.zpa), *SA = ZA + M;
+    if (M <= kDecodeMaxM) {
         GemvArgs g{};
         g.CA = CA; g.CB = CB; g.SCA = NDA; g.SCB = NDB;
         g.ZA = ZA; g.SA = SA; g.ZB = ZB; g.SB = SB;
@@ -337,6 +356,16 @@ int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K, const int8
     g.sk_partial = at<int32_t>(ws, L.sk);
     g.sk_flags = at<uint32_t>(ws, kWsSkFlagOffset);
     return from_cuda(launch_gemm_tc(g, s));
+}
+
+int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *NDB,
+                      const int32_t *ZB, const int32_t *SB, const void *bias, void *Y, void *ws, size_t ws_bytes,
+                      void *stream) {
+    int st = check_zp_weight_args(M, N, K, ZB, SB);
+    if (!st) st = check_forward_args(X, M, N, K, CB, NDB, nullptr, 0.f, bias, Y, true, true, ws, ws_bytes);
+    if (st) return st < 0 ? INT8LT_OK : st;
+    if ((st = int8lt_forward_zp_quantize(X, M, N, K, ws, ws_bytes, stream))) return st;
+    return int8lt_forward_zp_matmul(M, N, K, CB, NDB, ZB, SB, bias, Y, ws, ws_bytes, stream);
 }
 
 int int8lt_debug_gemm_i32(const int8_t *CA, const int8_t *CB, int64_t M, int64_t N, int64_t K, int32_t *C,

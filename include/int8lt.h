@@ -235,6 +235,21 @@ int int8lt_forward_zp(const void *X, int64_t M, int64_t N, int64_t K,
                       const int8_t *CB, const float *NDB, const int32_t *ZB, const int32_t *SB,
                       const void *bias, void *Y, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * The two halves of int8lt_forward_zp, as int8lt_forward_quantize /
+ * int8lt_forward_matmul are of int8lt_forward: int8lt_forward_zp is exactly
+ * _quantize then _matmul on the same stream and workspace.
+ *   _quantize: zeropoint codes, nd, zeropoints and code sums of X's rows
+ *              into the workspace (and, M <= 16, zeroes the GEMV's sums).
+ *   _matmul  : the int8 GEMM (M > 16) or GEMV (M <= 16) on those codes with
+ *              the zeropoint corrections, scales and bias fused, writing Y.
+ */
+int int8lt_forward_zp_quantize(const void *X, int64_t M, int64_t N, int64_t K,
+                               void *ws, size_t ws_bytes, void *stream);
+int int8lt_forward_zp_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, const float *NDB,
+                             const int32_t *ZB, const int32_t *SB, const void *bias, void *Y,
+                             void *ws, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------- tests -- */
 
 /*

@@ -100,6 +100,32 @@ def test_other_entry_validation(L):
     assert L.int8lt_read_device_status(FAKE, 16, None) == E["INT8LT_ERR_WORKSPACE"]
 
 
+def test_zeropoint_entry_validation(L):
+    E = _lib.STATUS_CODE
+    q = L.int8lt_quantize_rows_zp
+    assert q(None, 8, 64, FAKE, FAKE, FAKE, FAKE, None) == E["INT8LT_ERR_NULL"]
+    assert q(FAKE, 8, 64, FAKE, FAKE, None, FAKE, None) == E["INT8LT_ERR_NULL"]
+    assert q(FAKE, 8, 40, FAKE, FAKE, FAKE, FAKE, None) == E["INT8LT_ERR_SHAPE"]
+    assert q(FAKE + 8, 8, 64, FAKE, FAKE, FAKE, FAKE, None) == E["INT8LT_ERR_ALIGN"]
+    assert q(FAKE, 8, 64, FAKE + 4, FAKE, FAKE, FAKE, None) == E["INT8LT_ERR_ALIGN"]
+    assert q(FAKE, 0, 64, None, None, None, None, None) == E["INT8LT_OK"]   # empty: no-op
+    p = L.int8lt_prepare_weight_zp
+    assert p(FAKE, 12, 64, FAKE, FAKE, FAKE, FAKE, None) == E["INT8LT_ERR_SHAPE"]   # N % 8
+    ws = L.int8lt_workspace_size(32, 64, 64)
+    f = L.int8lt_forward_zp
+    assert f(FAKE, 32, 64, 64, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, ws, None) == E["INT8LT_ERR_NULL"]
+    assert f(FAKE, 32, 64, 64, FAKE, FAKE, FAKE + 2, FAKE, None, FAKE, FAKE, ws, None) == E["INT8LT_ERR_ALIGN"]
+    assert f(FAKE, 32, 64, 40, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, ws, None) == E["INT8LT_ERR_SHAPE"]
+    assert f(FAKE, 32, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 64, None) == E["INT8LT_ERR_WORKSPACE"]
+    assert f(FAKE, 0, 64, 64, None, None, None, None, None, None, None, 0, None) == E["INT8LT_OK"]
+    h = L.int8lt_forward_zp_quantize
+    assert h(None, 32, 64, 64, FAKE, ws, None) == E["INT8LT_ERR_NULL"]
+    assert h(FAKE, 32, 64, 64, FAKE, 64, None) == E["INT8LT_ERR_WORKSPACE"]
+    m = L.int8lt_forward_zp_matmul
+    assert m(32, 64, 64, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, ws, None) == E["INT8LT_ERR_NULL"]
+    assert m(32, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE + 8, FAKE, ws, None) == E["INT8LT_ERR_ALIGN"]
+
+
 def test_product_path_does_not_touch_oracle():
     pkg = os.path.join(ROOT, "bit_quantized_matmul_int8_b200")
     for dirpath, _, files in os.walk(pkg):

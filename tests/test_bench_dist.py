@@ -72,9 +72,28 @@ def test_reference_arm_other_ranks_print_nothing(capsys):
         steps = 1
         warmup = 0
         out = None
+        quant = "absmax"
 
     bench.run_reference(A, rank=1, world=2)
     assert capsys.readouterr().out == ""
     bench.run_reference(A, rank=0, world=2)
     line = capsys.readouterr().out.strip()
     assert line.startswith("{") and '"impl": "reference"' in line
+
+
+def test_reference_arm_zeropoint(capsys):
+    import json
+
+    import bench
+
+    class A:
+        workload = "tiny_16x64x64"
+        steps = 1
+        warmup = 0
+        out = None
+        quant = "zeropoint"
+
+    bench.run_reference(A, rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["config"]["quant"] == "zeropoint"
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"

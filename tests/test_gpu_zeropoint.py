@@ -142,6 +142,20 @@ def test_zp_forward_sampled_rows_large():
     check_y(Yg, Y64, w.name)
 
 
+@pytest.mark.parametrize("M", [5, 300])
+def test_zp_halves_equal_forward(M):
+    w = wl.random_case(84, M, 512, 264)
+    X = dev(asymmetric_rows(wl.make_x(w)))
+    b = dev(wl.make_bias(w))
+    CB, NDB, ZB, SB = _lib.int8lt_prepare_weight_zp(dev(wl.make_w(w)))
+    Y1 = _lib.int8lt_forward_zp(X, CB, NDB, ZB, SB, b)
+    ws = _lib.workspace(M, 264, 512, "cuda")
+    Y2 = torch.empty_like(Y1)
+    _lib.int8lt_forward_zp_quantize(X, 264, ws)
+    _lib.int8lt_forward_zp_matmul(M, CB, NDB, ZB, SB, b, Y2, ws)
+    assert torch.equal(Y1, Y2)
+
+
 def test_zp_forward_empty_and_errors():
     Xd = torch.zeros((0, 64), dtype=torch.float16, device="cuda")
     W = dev(wl.make_w(wl.random_case(83, 4, 64, 16)))
