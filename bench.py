@@ -309,9 +309,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     def fwd_matmul(CB, Y, ws, st):
         if zp:
-            _lib.int8lt_forward_zp_matmul(M, CB, NDB, ZB, SB, bd, Y, ws, st)
+            _lib.int8lt_forward_zp_matmul(M, K, CB, NDB, ZB, SB, bd, Y, ws, st)
         else:
-            _lib.int8lt_forward_matmul(M, CB, SCB, Wd, bd, Y, ws, st)
+            _lib.int8lt_forward_matmul(M, K, CB, SCB, Wd, bd, Y, ws, st)
 
     # Rotating input sets: X, CB, Y and workspace per set.
     ws_bytes = _lib.int8lt_workspace_size(M, N, K)

@@ -30,6 +30,7 @@ EXPORTS = [
     "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
     "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
     "int8lt_forward_zp_quantize", "int8lt_forward_zp_matmul",
+    "int8lt_weight_bytes", "int8lt_pack_weight", "int8lt_unpack_weight",
 ]
 
 
@@ -64,6 +65,9 @@ _SIGS = {
     "int8lt_prepare_weight_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "int8lt_forward_zp": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8lt_forward_zp_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "int8lt_weight_bytes": (_SZ, [_I64, _I64]),
+    "int8lt_pack_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "int8lt_unpack_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "int8lt_forward_zp_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
@@ -144,12 +148,50 @@ def workspace(M: int, N: int, K: int, device=None) -> torch.Tensor:
     return ws
 
 
+def blocked_weight(N: int, K: int, device=None) -> torch.Tensor:
+    """Uninitialised int8 buffer for [N,K] weight codes in the blocked weight layout:
+    shape [ceil(N/32), ceil(K/128), 32, 128] (row block, k-block, row, byte)."""
+    return torch.empty(((N + 31) // 32, (K + 127) // 128, 32, 128), dtype=torch.int8,
+                       device=device or "cuda")
+
+
+def _check_cb(CB: torch.Tensor, N: int, K: int) -> None:
+    _dev(CB, torch.int8, "CB")
+    if CB.numel() != int8lt_weight_bytes(N, K):
+        raise ValueError(f"CB holds {CB.numel()} bytes; the blocked codes of a [{N},{K}] weight "
+                         f"take {int8lt_weight_bytes(N, K)}")
+
+
+def int8lt_weight_bytes(N: int, K: int) -> int:
+    return int(lib().int8lt_weight_bytes(N, K))
+
+
+def int8lt_pack_weight(CB_rows: torch.Tensor, stream=None) -> torch.Tensor:
+    """Row-major int8 codes [N,K] -> the blocked weight layout."""
+    _dev(CB_rows, torch.int8, "CB_rows")
+    N, K = CB_rows.shape
+    CB = blocked_weight(N, K, CB_rows.device)
+    _check("int8lt_pack_weight",
+           lib().int8lt_pack_weight(_ptr(CB_rows), N, K, _ptr(CB), _stream(stream)))
+    return CB
+
+
+def int8lt_unpack_weight(CB: torch.Tensor, N: int, K: int, stream=None) -> torch.Tensor:
+    """Blocked weight codes -> row-major int8 [N,K]."""
+    _check_cb(CB, N, K)
+    rows = torch.empty((N, K), dtype=torch.int8, device=CB.device)
+    _check("int8lt_unpack_weight",
+           lib().int8lt_unpack_weight(_ptr(CB), N, K, _ptr(rows), _stream(stream)))
+    return rows
+
+
 def int8lt_prepare_weight(W: torch.Tensor, CB: torch.Tensor | None = None,
                           SCB: torch.Tensor | None = None, stream=None):
-    """W fp16 [N,K] -> (CB int8 [N,K], SCB fp32 [N])."""
+    """W fp16 [N,K] -> (CB int8, blocked weight layout, SCB fp32 [N])."""
     _dev(W, torch.float16, "W")
     N, K = W.shape
-    CB = torch.empty((N, K), dtype=torch.int8, device=W.device) if CB is None else CB
+    CB = blocked_weight(N, K, W.device) if CB is None else CB
+    _check_cb(CB, N, K)
     SCB = torch.empty(N, dtype=torch.float32, device=W.device) if SCB is None else SCB
     _check("int8lt_prepare_weight",
            lib().int8lt_prepare_weight(_ptr(W), N, K, _ptr(CB), _ptr(SCB), _stream(stream)))
@@ -180,14 +222,14 @@ def int8lt_forward(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
                    ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Y fp16 [M,N] = LLM.int8() forward of X fp16 [M,K] with CB/SCB (and fp16 outlier weights)."""
     _dev(X, torch.float16, "X")
-    _dev(CB, torch.int8, "CB")
     _dev(SCB, torch.float32, "SCB")
     if W_outlier is not None:
         _dev(W_outlier, torch.float16, "W_outlier")
     if bias is not None:
         _dev(bias, torch.float16, "bias")
     M, K = X.shape
-    N = CB.shape[0]
+    N = SCB.shape[0]
+    _check_cb(CB, N, K)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
     if ws is None:
@@ -204,17 +246,17 @@ def int8lt_forward_quantize(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor
                             stream=None) -> None:
     """First half of int8lt_forward: quantize X (and gather outlier weights) into ws."""
     M, K = X.shape
-    N = CB.shape[0]
+    N = SCB.shape[0]
     _check("int8lt_forward_quantize",
            lib().int8lt_forward_quantize(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier),
                                          float(threshold), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def int8lt_forward_matmul(M: int, CB: torch.Tensor, SCB: torch.Tensor,
+def int8lt_forward_matmul(M: int, K: int, CB: torch.Tensor, SCB: torch.Tensor,
                           W_outlier: torch.Tensor | None, bias: torch.Tensor | None,
                           Y: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
     """Second half of int8lt_forward: GEMM/GEMV + fused epilogue from ws into Y."""
-    N, K = CB.shape
+    N = SCB.shape[0]
     _check("int8lt_forward_matmul",
            lib().int8lt_forward_matmul(M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier), _ptr(bias),
                                        _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
@@ -232,7 +274,7 @@ def int8lt_forward_static_scratch(X: torch.Tensor, CB: torch.Tensor, SCB: torch.
     overlap on the GPU share the one array and race; order them on one stream.
     """
     M, K = X.shape
-    N = CB.shape[0]
+    N = SCB.shape[0]
     _check("int8lt_forward_static_scratch",
            lib().int8lt_forward_static_scratch(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB),
                                                _ptr(W_outlier), float(threshold), _ptr(bias),
@@ -240,12 +282,12 @@ def int8lt_forward_static_scratch(X: torch.Tensor, CB: torch.Tensor, SCB: torch.
     return Y
 
 
-def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, ws: torch.Tensor | None = None,
+def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, N: int, ws: torch.Tensor | None = None,
                           stream=None) -> torch.Tensor:
+    """int32 CA [M,K] . CB^T with CB in the blocked weight layout (see int8lt_pack_weight)."""
     _dev(CA, torch.int8, "CA")
-    _dev(CB, torch.int8, "CB")
     M, K = CA.shape
-    N = CB.shape[0]
+    _check_cb(CB, N, K)
     C = torch.empty((M, N), dtype=torch.int32, device=CA.device)
     if ws is None:
         ws = workspace(M, N, K, CA.device)
@@ -260,7 +302,7 @@ def int8lt_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> N
            lib().int8lt_debug_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
 
 
-def int8lt_quantize_rows_zp(X: torch.Tensor, stream=None, _fn: str = "int8lt_quantize_rows_zp"):
+def int8lt_quantize_rows_zp(X: torch.Tensor, stream=None):
     """Zeropoint quantization of each row of X fp16 [R,K] -> (Q int8 [R,K], ND fp32 [R],
     ZP int32 [R], SUM int32 [R])."""
     _dev(X, torch.float16, "X")
@@ -270,14 +312,26 @@ def int8lt_quantize_rows_zp(X: torch.Tensor, stream=None, _fn: str = "int8lt_qua
     ND = torch.empty(R, dtype=torch.float32, device=dev)
     ZP = torch.empty(R, dtype=torch.int32, device=dev)
     SUM = torch.empty(R, dtype=torch.int32, device=dev)
-    _check(_fn, getattr(lib(), _fn)(_ptr(X), R, K, _ptr(Q), _ptr(ND), _ptr(ZP), _ptr(SUM),
-                                    _stream(stream)))
+    _check("int8lt_quantize_rows_zp",
+           lib().int8lt_quantize_rows_zp(_ptr(X), R, K, _ptr(Q), _ptr(ND), _ptr(ZP), _ptr(SUM),
+                                         _stream(stream)))
     return Q, ND, ZP, SUM
 
 
 def int8lt_prepare_weight_zp(W: torch.Tensor, stream=None):
-    """W fp16 [N,K] -> (CB int8 [N,K], NDB fp32 [N], ZB int32 [N], SB int32 [N])."""
-    return int8lt_quantize_rows_zp(W, stream, "int8lt_prepare_weight_zp")
+    """W fp16 [N,K] -> (CB int8 in the blocked weight layout, NDB fp32 [N], ZB int32 [N],
+    SB int32 [N])."""
+    _dev(W, torch.float16, "W")
+    N, K = W.shape
+    dev = W.device
+    CB = blocked_weight(N, K, dev)
+    NDB = torch.empty(N, dtype=torch.float32, device=dev)
+    ZB = torch.empty(N, dtype=torch.int32, device=dev)
+    SB = torch.empty(N, dtype=torch.int32, device=dev)
+    _check("int8lt_prepare_weight_zp",
+           lib().int8lt_prepare_weight_zp(_ptr(W), N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
+                                          _stream(stream)))
+    return CB, NDB, ZB, SB
 
 
 def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: torch.Tensor,
@@ -286,14 +340,14 @@ def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: 
                       stream=None) -> torch.Tensor:
     """Y fp16 [M,N]: zeropoint-quantized X times the zeropoint-quantized weight, plus bias."""
     _dev(X, torch.float16, "X")
-    _dev(CB, torch.int8, "CB")
     _dev(NDB, torch.float32, "NDB")
     _dev(ZB, torch.int32, "ZB")
     _dev(SB, torch.int32, "SB")
     if bias is not None:
         _dev(bias, torch.float16, "bias")
     M, K = X.shape
-    N = CB.shape[0]
+    N = NDB.shape[0]
+    _check_cb(CB, N, K)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
     if ws is None:
@@ -311,11 +365,11 @@ def int8lt_forward_zp_quantize(X: torch.Tensor, N: int, ws: torch.Tensor, stream
            lib().int8lt_forward_zp_quantize(_ptr(X), M, N, K, _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def int8lt_forward_zp_matmul(M: int, CB: torch.Tensor, NDB: torch.Tensor, ZB: torch.Tensor,
+def int8lt_forward_zp_matmul(M: int, K: int, CB: torch.Tensor, NDB: torch.Tensor, ZB: torch.Tensor,
                              SB: torch.Tensor, bias: torch.Tensor | None, Y: torch.Tensor,
                              ws: torch.Tensor, stream=None) -> None:
     """Second half of int8lt_forward_zp: GEMM/GEMV with the zeropoint epilogue into Y."""
-    N, K = CB.shape
+    N = NDB.shape[0]
     _check("int8lt_forward_zp_matmul",
            lib().int8lt_forward_zp_matmul(M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
                                           _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(),

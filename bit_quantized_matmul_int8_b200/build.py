@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["api.cu", "quantize.cu", "gemm_tc.cu", "gemv.cu", "static_scratch.cu",
-           "zeropoint.cu"]
+           "zeropoint.cu", "weight_layout.cu"]
 LIB = os.path.join(HERE, "libint8lt.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",

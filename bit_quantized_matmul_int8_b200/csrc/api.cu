@@ -223,6 +223,31 @@ int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream) {
     return (status & kStatusTimeout) ? INT8LT_ERR_TIMEOUT : INT8LT_ERR_CUDA;
 }
 
+size_t int8lt_weight_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K < 1 || K > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return 0;
+    return (size_t)weight_bytes(N, K);
+}
+
+static int convert_weight(bool pack, const int8_t *src, int64_t N, int64_t K, int8_t *dst, void *stream) {
+    if (N < 0 || K < 1 || K > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return INT8LT_ERR_SHAPE;
+    if (N == 0) return INT8LT_OK;
+    if (!src || !dst) return INT8LT_ERR_NULL;
+    const int8_t *blocked = pack ? dst : src;
+    const int8_t *rows = pack ? src : dst;
+    if (!aligned(blocked, 16) || ((K % 16) == 0 && !aligned(rows, 16))) return INT8LT_ERR_ALIGN;
+    if (int st = check_device()) return st;
+    return from_cuda(launch_convert_weight(pack, const_cast<int8_t *>(blocked), const_cast<int8_t *>(rows), N, K,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int int8lt_pack_weight(const int8_t *CB_rows, int64_t N, int64_t K, int8_t *CB, void *stream) {
+    return convert_weight(true, CB_rows, N, K, CB, stream);
+}
+
+int int8lt_unpack_weight(const int8_t *CB, int64_t N, int64_t K, int8_t *CB_rows, void *stream) {
+    return convert_weight(false, CB, N, K, CB_rows, stream);
+}
+
 int int8lt_prepare_weight(const void *W, int64_t N, int64_t K, int8_t *CB, float *SCB, void *stream) {
     if (!W || !CB || !SCB) return INT8LT_ERR_NULL;
     if (N < 0 || K < 1 || K > ((int64_t)1 << 31)) return INT8LT_ERR_SHAPE;
@@ -304,7 +329,15 @@ int int8lt_quantize_rows_zp(const void *X, int64_t R, int64_t K, int8_t *Q, floa
 int int8lt_prepare_weight_zp(const void *W, int64_t N, int64_t K, int8_t *CB, float *NDB, int32_t *ZB,
                              int32_t *SB, void *stream) {
     if (!shape_ok(8, N, K)) return INT8LT_ERR_SHAPE;
-    return int8lt_quantize_rows_zp(W, N, K, CB, NDB, ZB, SB, stream);
+    if (N == 0) return INT8LT_OK;
+    if (!W || !CB || !NDB || !ZB || !SB) return INT8LT_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(CB, 16) || !aligned(NDB, 4) || !aligned(ZB, 4) || !aligned(SB, 4))
+        return INT8LT_ERR_ALIGN;
+    if (int st = check_device()) return st;
+    ZpQuantArgs z{};
+    z.X = static_cast<const __half *>(W); z.R = N; z.K = K;
+    z.Q = CB; z.blocked = true; z.ND = NDB; z.ZP = ZB; z.SUM = SB;
+    return from_cuda(launch_zp_quantize(z, static_cast<cudaStream_t>(stream)));
 }
 
 int int8lt_forward_zp_quantize(const void *X, int64_t M, int64_t N, int64_t K, void *ws, size_t ws_bytes,

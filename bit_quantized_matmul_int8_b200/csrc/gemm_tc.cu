@@ -445,7 +445,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     if (rank == 0) mbar_arrive_expect_tx(fb, kTxBytes);
                     const uint32_t fb_leader = mapa_shared(fb, 0);
                     tma_load_2d_pair(smem_u32(sA + stage * kStageA), &tmA, fb_leader, kb * 128, m0);
-                    tma_load_2d_pair(smem_u32(sB + stage * kStageB), &tmB, fb_leader, kb * 128, n0);
+                    tma_load_4d_pair(smem_u32(sB + stage * kStageB), &tmB, fb_leader, 0, 0, kb,
+                                     (int32_t)(n0 / kWBlockRows));
                     ++issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
@@ -786,6 +787,23 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t
 }
 
 namespace {
+// CB in the blocked weight layout as a 4-D tensor (128 bytes, 32 rows,
+// k-blocks, row blocks); a box of (128, 32, 1, 4) is one k-block of 128
+// consecutive output channels, landing in shared memory exactly as a 128-row
+// x 128-byte box of a row-major matrix would (same 128-byte swizzle).
+bool make_map_wblocks(CUtensorMap *m, const int8_t *CB, int64_t N, int64_t K) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const int64_t KB = wblocks_k(K), NB = ceil_div(N, kWBlockRows);
+    cuuint64_t dims[4] = {(cuuint64_t)kWBlockCols, (cuuint64_t)kWBlockRows, (cuuint64_t)KB, (cuuint64_t)NB};
+    cuuint64_t strides[3] = {(cuuint64_t)kWBlockCols, (cuuint64_t)kWBlockBytes, (cuuint64_t)(KB * kWBlockBytes)};
+    cuuint32_t box[4] = {(cuuint32_t)kWBlockCols, (cuuint32_t)kWBlockRows, 1, kCtaRows / kWBlockRows};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<int8_t *>(CB), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int g_num_sms[64];  // resident CTA pairs per device
 
 }  // namespace
@@ -793,7 +811,7 @@ int g_num_sms[64];  // resident CTA pairs per device
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s) {
     CUtensorMap mA, mB, mXo, mWo;
     if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CA, a.K, a.M, a.K, 128, kCtaRows) ||
-        !make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.CB, a.K, a.N, a.K, 128, kCtaRows))
+        !make_map_wblocks(&mB, a.CB, a.N, a.K))
         return cudaErrorInvalidValue;
     if (a.Xo && a.Wo && a.n_outliers) {
         if (!make_map(&mXo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Xo, a.kcap, a.M, a.kcap * 2, kOkb, kCtaRows,

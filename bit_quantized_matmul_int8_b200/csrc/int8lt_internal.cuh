@@ -22,6 +22,21 @@ constexpr uint32_t kStatusTimeout = 1u;
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
+// Weight codes (CB) are stored in blocks of 32 output channels x 128 bytes of
+// K, each block 4 KB contiguous, blocks ordered by row block, then k-block:
+//   CB[j, k] at ((j / 32) * ceil(K / 128) + k / 128) * 4096 + (j % 32) * 128 + k % 128.
+// Codes past N rows or K columns inside the last blocks are zero. A decode
+// GEMV then streams one contiguous range of CB per warp, and the GEMM's TMA
+// reads a 128-row tile as four 4 KB blocks.
+constexpr int64_t kWBlockRows = 32, kWBlockCols = 128, kWBlockBytes = kWBlockRows * kWBlockCols;
+__host__ __device__ __forceinline__ int64_t wblocks_k(int64_t K) { return ceil_div(K, kWBlockCols); }
+__host__ __device__ __forceinline__ int64_t cb_offset(int64_t j, int64_t k, int64_t KB) {
+    return ((j >> 5) * KB + (k >> 7)) * kWBlockBytes + (j & 31) * kWBlockCols + (k & 127);
+}
+__host__ __device__ __forceinline__ int64_t weight_bytes(int64_t N, int64_t K) {
+    return ceil_div(N, kWBlockRows) * wblocks_k(K) * kWBlockBytes;
+}
+
 // Byte offsets of the workspace sections (every section 1024-byte aligned).
 // The header and the two column bitmaps sit at fixed offsets whatever the
 // shape, so one zeroing of the first kWsInitBytes prepares any workspace.
@@ -58,6 +73,9 @@ static_assert(2 * kSkMaxPairs * 4 <= 1024, "stream-K flags");
 // fp16 bit pattern T: |x| >= threshold  <=>  (bits(x) & 0x7fff) >= T.
 uint16_t threshold_bits(float threshold);
 
+// Row-major int8 codes [N, K] <-> the blocked weight layout (pack: rows -> blocked).
+cudaError_t launch_convert_weight(bool pack, int8_t *blocked, int8_t *rows, int64_t N, int64_t K, cudaStream_t s);
+
 cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
                                   cudaStream_t s);
 
@@ -93,7 +111,8 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s);
 struct ZpQuantArgs {
     const __half *X;
     int64_t R, K;
-    int8_t *Q;                // [R, K] codes
+    int8_t *Q;                // [R, K] codes, row-major (or the blocked weight layout)
+    bool blocked;             // Q in the blocked weight layout, padding zeroed
     float *ND;                // [R]
     int32_t *ZP;              // [R]
     int32_t *SUM;             // [R]
@@ -373,6 +392,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 4-D tiled TMA load (coordinates innermost first) into this CTA's shared
+// memory, completion counted on the mbarrier at `bar_cluster` as for
+// tma_load_2d_pair. No multicast.
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap *m, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
 }
 
 // 2-D tiled TMA load into this CTA's shared memory whose completion is

@@ -86,28 +86,35 @@ prepare_weight_kernel(const __half *__restrict__ W, int64_t N, int64_t K, int8_t
     const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
     const bool vec = (K % 8) == 0;
-    for (int64_t j = warp; j < N; j += nwarps) {
-        const __half *w = W + j * K;
-        int8_t *cb = CB + j * K;
-        uint32_t amax = 0;
-        if (vec) {
-            const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
-            for (int64_t v = lane; v < K / 8; v += 32) amax = max(amax, vec_absmax_bits(__ldg(w4 + v)));
-        } else {
-            const uint16_t *wb = reinterpret_cast<const uint16_t *>(w);
-            for (int64_t k = lane; k < K; k += 32) amax = max(amax, (uint32_t)(wb[k] & 0x7fffu));
+    const int64_t KB = wblocks_k(K), Kp = KB * kWBlockCols;
+    // Rows past N inside the last row block are written as zero codes.
+    for (int64_t j = warp; j < round_up(N, kWBlockRows); j += nwarps) {
+        int64_t kz = 0;  // first column written as zero padding
+        if (j < N) {
+            const __half *w = W + j * K;
+            uint32_t amax = 0;
+            if (vec) {
+                const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
+                for (int64_t v = lane; v < K / 8; v += 32) amax = max(amax, vec_absmax_bits(__ldg(w4 + v)));
+            } else {
+                const uint16_t *wb = reinterpret_cast<const uint16_t *>(w);
+                for (int64_t k = lane; k < K; k += 32) amax = max(amax, (uint32_t)(wb[k] & 0x7fffu));
+            }
+            amax = warp_max_u32(amax);
+            const float a = __half2float(__ushort_as_half((unsigned short)amax));
+            const float s = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+            if (vec) {
+                const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
+                for (int64_t v = lane; v < K / 8; v += 32)
+                    *reinterpret_cast<uint2 *>(CB + cb_offset(j, v * 8, KB)) = quant_vec8(__ldg(w4 + v), s);
+            } else {
+                for (int64_t k = lane; k < K; k += 32)
+                    CB[cb_offset(j, k, KB)] = (int8_t)(code_bits(__half2float(w[k]), s) & 0xffu);
+            }
+            if (lane == 0) SCB[j] = a;
+            kz = K;
         }
-        amax = warp_max_u32(amax);
-        const float a = __half2float(__ushort_as_half((unsigned short)amax));
-        const float s = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-        if (vec) {
-            const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
-            uint2 *c2 = reinterpret_cast<uint2 *>(cb);
-            for (int64_t v = lane; v < K / 8; v += 32) c2[v] = quant_vec8(__ldg(w4 + v), s);
-        } else {
-            for (int64_t k = lane; k < K; k += 32) cb[k] = (int8_t)(code_bits(__half2float(w[k]), s) & 0xffu);
-        }
-        if (lane == 0) SCB[j] = a;
+        for (int64_t k = kz + lane; k < Kp; k += 32) CB[cb_offset(j, k, KB)] = 0;
     }
 }
 
@@ -463,7 +470,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
                 if (a.W_outlier) {
                     gv[u] = a.W_outlier[j * a.K + col];
                 } else {
-                    const float p = __fmul_rn((float)a.CB[j * a.K + col], a.SCB[j]);
+                    const float p = __fmul_rn((float)a.CB[cb_offset(j, col, wblocks_k(a.K))], a.SCB[j]);
                     gv[u] = __float2half_rn(__fdiv_rn(p, 127.f));
                 }
             }
@@ -566,7 +573,7 @@ uint16_t threshold_bits(float threshold) {
 
 cudaError_t launch_prepare_weight(const __half *W, int64_t N, int64_t K, int8_t *CB, float *SCB,
                                   cudaStream_t s) {
-    int64_t blocks = ceil_div(N, kWarps);
+    int64_t blocks = ceil_div(round_up(N, kWBlockRows), kWarps);
     if (blocks > 148 * 16) blocks = 148 * 16;
     prepare_weight_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(W, N, K, CB, SCB);
     return cudaGetLastError();

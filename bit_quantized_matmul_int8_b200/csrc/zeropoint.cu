@@ -11,8 +11,10 @@
 // the codes the pass writes nd, zp and the sum of the row's codes, the three
 // per-row terms that the unrolled product (A + zp_a)(B + zp_b) needs.
 //
-// One CTA (8 warps) per row for long rows or few rows, one warp per row
-// otherwise; rows are read twice with 16-byte loads (min/max, then codes),
+// Weight rows (output channels) are written in the blocked weight layout
+// (4 KB blocks of 32 rows x 128 bytes, padding zeroed), activation rows
+// row-major. One CTA (8 warps) per row for long rows or few rows, one warp
+// per row otherwise; rows are read twice with 16-byte loads (min/max, then codes),
 // the second time mostly from L1. The pass also zeroes the decode GEMV's
 // partial sums and counters when asked, as the absmax quantize pass does.
 #include <algorithm>
@@ -75,6 +77,14 @@ __global__ void __launch_bounds__(kThreads) zp_quantize_kernel(const ZpQuantArgs
         if (a.cnt)
             for (int64_t i = tid; i < a.cnt_words / 4; i += nth)
                 reinterpret_cast<uint4 *>(a.cnt)[i] = make_uint4(0, 0, 0, 0);
+        // Blocked weight layout: rows past R inside the last row block are zero codes.
+        if (a.blocked) {
+            const int64_t KB = wblocks_k(a.K), per_row = KB * kWBlockCols / 16;
+            const int64_t pad = (round_up(a.R, kWBlockRows) - a.R) * per_row;
+            for (int64_t i = tid; i < pad; i += nth)
+                *reinterpret_cast<uint4 *>(a.Q + cb_offset(a.R + i / per_row, (i % per_row) * 16, KB)) =
+                    make_uint4(0, 0, 0, 0);
+        }
     }
 
     const int64_t nvec = a.K / 8;
@@ -115,9 +125,16 @@ __global__ void __launch_bounds__(kThreads) zp_quantize_kernel(const ZpQuantArgs
 
         // Pass 2: codes and their sum.
         int32_t sum = 0;
-        if (live)
+        if (live && a.blocked) {
+            const int64_t KB = wblocks_k(a.K);
+            for (int64_t v = t; v < nvec; v += kLanes)
+                *reinterpret_cast<uint2 *>(a.Q + cb_offset(row, v * 8, KB)) = codes8(ld_row(x + v * 8), nd, zp, sum);
+            for (int64_t v = nvec + t; v < KB * kWBlockCols / 8; v += kLanes)  // padding columns
+                *reinterpret_cast<uint2 *>(a.Q + cb_offset(row, v * 8, KB)) = make_uint2(0u, 0u);
+        } else if (live) {
             for (int64_t v = t; v < nvec; v += kLanes)
                 *reinterpret_cast<uint2 *>(a.Q + row * a.K + v * 8) = codes8(ld_row(x + v * 8), nd, zp, sum);
+        }
 #pragma unroll
         for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if constexpr (kWarpsPerRow > 1) {
@@ -142,7 +159,8 @@ cudaError_t launch_zp_quantize(const ZpQuantArgs &a, cudaStream_t s) {
     if (a.R <= 0) return cudaSuccess;
     const bool per_cta = a.K >= 2048 || a.R < 4 * 148;
     const int64_t groups = per_cta ? a.R : ceil_div(a.R, kWarps);
-    const int64_t clear = ceil_div((a.acc ? a.acc_words : 0) + (a.cnt ? a.cnt_words : 0), 4 * kThreads);
+    const int64_t pad = a.blocked ? (round_up(a.R, kWBlockRows) - a.R) * wblocks_k(a.K) * kWBlockCols / 4 : 0;
+    const int64_t clear = ceil_div((a.acc ? a.acc_words : 0) + (a.cnt ? a.cnt_words : 0) + pad, 4 * kThreads);
     int64_t grid = std::max<int64_t>(groups, std::min<int64_t>(clear, 148 * 4));
     grid = std::min<int64_t>(grid, (int64_t)1 << 20);
     if (per_cta)

@@ -21,8 +21,16 @@
  *         Decomposition" (threshold alpha = 6.0).
  *
  * Conventions for every entry point:
- *   - Matrices are dense row-major. X is [M, K] (tokens x features), W and CB
- *     are [N, K] (nn.Linear layout: one row per output channel), Y is [M, N].
+ *   - Matrices are dense row-major. X is [M, K] (tokens x features), W is
+ *     [N, K] (nn.Linear layout: one row per output channel), Y is [M, N].
+ *   - The int8 weight codes CB, logically [N, K], are stored in this
+ *     library's blocked weight layout: 4096-byte blocks of 32 output channels
+ *     x 128 bytes of K, ordered row block by row block (k-blocks inside),
+ *     each block row-major; CB[j, k] sits at byte
+ *       ((j / 32) * ceil(K / 128) + k / 128) * 4096 + (j % 32) * 128 + k % 128,
+ *     and the codes past N or K inside the last blocks are zero. The buffer
+ *     has int8lt_weight_bytes(N, K) bytes. int8lt_pack_weight and
+ *     int8lt_unpack_weight convert from and to row-major codes.
  *   - "fp16" means IEEE binary16, passed as void pointers. Every tensor
  *     pointer is DEVICE memory owned by the caller; the library allocates
  *     nothing and keeps no per-call state. `stream` is a cudaStream_t (NULL =
@@ -102,7 +110,23 @@ int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream);
 int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Weight conversion: W fp16 [N, K] -> CB int8 [N, K] and SCB fp32 [N].
+ * Bytes of the blocked weight codes of an [N, K] weight:
+ * ceil(N / 32) * ceil(K / 128) * 4096. Returns 0 for N < 0 or K < 1.
+ */
+size_t int8lt_weight_bytes(int64_t N, int64_t K);
+
+/*
+ * Layout conversions (stream-ordered): row-major int8 codes CB_rows [N, K]
+ * -> the blocked weight layout CB (int8lt_weight_bytes(N, K) bytes, padding
+ * written as zero), and back (only the N x K codes are written). CB must be
+ * 16-byte aligned, CB_rows too when K % 16 == 0. Any N >= 0, K >= 1.
+ */
+int int8lt_pack_weight(const int8_t *CB_rows, int64_t N, int64_t K, int8_t *CB, void *stream);
+int int8lt_unpack_weight(const int8_t *CB, int64_t N, int64_t K, int8_t *CB_rows, void *stream);
+
+/*
+ * Weight conversion: W fp16 [N, K] -> CB int8 [N, K] (blocked weight
+ * layout, int8lt_weight_bytes(N, K) bytes) and SCB fp32 [N].
  * [HF] "transformers integration": weights become int8 in [-127, 127] with a
  * per-output-channel scale, recoverable as W ~= CB * SCB / 127; [P] absmax
  * equation, vector-wise (per output channel). SCB[j] = max_k |W[j,k]|,
@@ -137,7 +161,7 @@ int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold,
  * vector-wise equations), O and CA/SCA as in int8lt_quantize_rows, and the
  * outlier term of [P] "Mixed-precision Decomposition" / [HF] step 3.
  * The combination is computed in fp32 and rounded once to fp16.
- *   CB, SCB   : from int8lt_prepare_weight.
+ *   CB, SCB   : from int8lt_prepare_weight (CB in the blocked weight layout).
  *   W_outlier : fp16 [N, K] weights for the outlier columns (only the columns
  *               in O are read), or NULL to use fp16(fp32(CB * SCB) / 127).
  *   bias      : fp16 [N] or NULL.
@@ -207,10 +231,11 @@ int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N, int64_t K
  * page's zeropoint formula is garbled; this is the reading whose shifted
  * codes the page's product (A + zp_a)(B + zp_b) takes. Unlike absmax codes,
  * the full [-127, 127] range is used by every row whatever its sign balance.
- *   Q   : int8 [R, K] (16-byte aligned); ND fp32 [R]; ZP, SUM int32 [R].
+ *   Q   : int8 [R, K] row-major (16-byte aligned); ND fp32 [R]; ZP, SUM int32 [R].
  * K % 16 == 0, 16 <= K <= 133144 (as for int8lt_forward). Deterministic; no
  * workspace. int8lt_prepare_weight_zp is the same operation on W [N, K]
- * (N % 8 == 0), written CB / NDB / ZB / SB for int8lt_forward_zp.
+ * (N % 8 == 0), written CB / NDB / ZB / SB for int8lt_forward_zp, with CB in
+ * the blocked weight layout (int8lt_weight_bytes(N, K) bytes).
  */
 int int8lt_quantize_rows_zp(const void *X, int64_t R, int64_t K, int8_t *Q, float *ND,
                             int32_t *ZP, int32_t *SUM, void *stream);
@@ -253,7 +278,8 @@ int int8lt_forward_zp_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, 
 /* ---------------------------------------------------------------- tests -- */
 
 /*
- * Test entry: the int8 GEMM alone, C int32 [M, N] = CA [M, K] . CB [N, K]^T,
+ * Test entry: the int8 GEMM alone, C int32 [M, N] = CA [M, K] . CB [N, K]^T
+ * (CA row-major, CB in the blocked weight layout),
  * through the same kernels int8lt_forward dispatches to (M <= 16: the GEMV,
  * otherwise the tcgen05 GEMM) with the dequantizing epilogue replaced by an
  * int32 store, so the accumulators can be compared bit for bit. Same shape,

@@ -80,17 +80,19 @@ def test_full_size_config(name):
     assert np.array_equal(host(CA), CAo)
 
     # CB / SCB on sampled weight rows
+    CBrows = _lib.int8lt_unpack_weight(CB, w.N, w.K)
     jr = _sample_rows(w.N, 64, 1)
     CBo, SCBo = oracle.prepare_weight(W[jr])
-    assert np.array_equal(host(CB[torch.from_numpy(jr).cuda()]), CBo)
+    assert np.array_equal(host(CBrows[torch.from_numpy(jr).cuda()]), CBo)
     assert np.array_equal(host(SCB[torch.from_numpy(jr).cuda()]), SCBo)
 
     # int32 accumulators on sampled rows (same kernel as the forward's matmul)
     rows = _sample_rows(w.M, 3 if w.M * w.N * w.K > 1e12 else 6, 2)
-    C = _lib.int8lt_debug_gemm_i32(CA, CB, ws=ws)
+    C = _lib.int8lt_debug_gemm_i32(CA, CB, w.N, ws=ws)
     Cs = host(C[torch.from_numpy(rows).cuda()])
     del C
-    CBfull = host(CB)
+    CBfull = host(CBrows)
+    del CBrows
     Cref = oracle.gemm_i32(CAo[rows], CBfull)
     assert np.array_equal(Cs, Cref)
 

@@ -23,6 +23,11 @@ def _built():
     ensure_built()
 
 
+def gemm_i32_gpu(A: np.ndarray, B: np.ndarray) -> torch.Tensor:
+    """int32 A . B^T through the GEMM / GEMV, B packed into the blocked weight layout."""
+    return _lib.int8lt_debug_gemm_i32(dev(A), _lib.int8lt_pack_weight(dev(B)), B.shape[0])
+
+
 # ------------------------------------------------------------ weight prep --
 
 @pytest.mark.parametrize("N,K", [(64, 64), (200, 4096), (24, 40), (8, 3), (513, 1000)])
@@ -32,8 +37,25 @@ def test_prepare_weight_bit_exact(N, K):
     W[N // 2] = 0                                   # all-zero channel: scale 0
     CB, SCB = _lib.int8lt_prepare_weight(dev(W))
     CBo, SCBo = oracle.prepare_weight(W)
-    assert np.array_equal(host(CB), CBo)
+    assert np.array_equal(host(_lib.int8lt_unpack_weight(CB, N, K)), CBo)
     assert np.array_equal(host(SCB).view(np.uint32), SCBo.view(np.uint32))
+    # the blocked layout's padding (rows past N, columns past K) holds zero codes
+    assert torch.equal(_lib.int8lt_pack_weight(dev(CBo)), CB)
+
+
+@pytest.mark.parametrize("N,K", [(8, 16), (40, 136), (96, 4096), (33, 7), (64, 250)])
+def test_weight_layout_roundtrip(N, K):
+    rng = np.random.default_rng(N * 1000 + K)
+    rows = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    CB = _lib.int8lt_pack_weight(dev(rows))
+    assert CB.numel() == _lib.int8lt_weight_bytes(N, K) == -(-N // 32) * -(-K // 128) * 4096
+    blk = host(CB).reshape(-(-N // 32), -(-K // 128), 32, 128)
+    for j, k in [(0, 0), (N - 1, K - 1), (N // 2, K // 3), (min(N - 1, 31), min(K - 1, 127))]:
+        assert blk[j // 32, k // 128, j % 32, k % 128] == rows[j, k]
+    full = np.zeros((blk.shape[0] * 32, blk.shape[1] * 128), np.int8)
+    full[:N, :K] = rows
+    assert np.array_equal(blk.transpose(0, 2, 1, 3).reshape(full.shape), full)
+    assert np.array_equal(host(_lib.int8lt_unpack_weight(CB, N, K)), rows)
 
 
 def test_prepare_weight_idempotent():
@@ -111,7 +133,7 @@ def test_gemm_int32_bit_exact(M, N, K):
     if M > 2:
         A[1] = 127
         B[0] = -127 if N > 1 else B[0]
-    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    C = host(gemm_i32_gpu(A, B))
     ref = A.astype(np.int64) @ B.astype(np.int64).T          # exact in int64
     assert np.array_equal(C.astype(np.int64), ref)
 
@@ -133,7 +155,7 @@ def test_gemm_int32_split_tiles_bit_exact(M, N, K, split_always):
     rng = np.random.default_rng(M + N + K)
     A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
     B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
-    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    C = host(gemm_i32_gpu(A, B))
     assert np.array_equal(C, oracle.gemm_i32(A, B))
 
 
@@ -143,7 +165,7 @@ def test_gemm_int32_split_auto_sampled_rows():
     rng = np.random.default_rng(76)
     A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
     B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
-    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    C = host(gemm_i32_gpu(A, B))
     rows = np.array([0, 1, 255, 256, 300, 511, 512, 700, 767, 768, 1000, 1023])
     assert np.array_equal(C[rows], oracle.gemm_i32(A[rows], B))
 
@@ -152,7 +174,7 @@ def test_gemm_int32_matches_oracle_routine():
     rng = np.random.default_rng(9)
     A = rng.integers(-127, 128, (200, 336), dtype=np.int64).astype(np.int8)
     B = rng.integers(-127, 128, (264, 336), dtype=np.int64).astype(np.int8)
-    assert np.array_equal(host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B))), oracle.gemm_i32(A, B))
+    assert np.array_equal(host(gemm_i32_gpu(A, B)), oracle.gemm_i32(A, B))
 
 
 def test_gemm_int32_extreme_k():
@@ -160,7 +182,7 @@ def test_gemm_int32_extreme_k():
     K = 133136
     A = np.full((20, K), 127, np.int8)
     B = np.full((8, K), -127, np.int8)
-    C = host(_lib.int8lt_debug_gemm_i32(dev(A), dev(B)))
+    C = host(gemm_i32_gpu(A, B))
     assert (C.astype(np.int64) == -127 * 127 * K).all()
 
 
@@ -307,6 +329,6 @@ def test_split_halves_equal_forward():
         ws = _lib.workspace(w.M, w.N, w.K)
         y2 = torch.empty_like(y1)
         _lib.int8lt_forward_quantize(Xd, CB, SCB, Wd, 6.0, ws)
-        _lib.int8lt_forward_matmul(w.M, CB, SCB, Wd, bd, y2, ws)
+        _lib.int8lt_forward_matmul(w.M, w.K, CB, SCB, Wd, bd, y2, ws)
         torch.cuda.synchronize()
         assert torch.equal(y1, y2)

@@ -74,10 +74,14 @@ def test_zp_quantize_rows_bit_exact(name, R, K):
     check_zp_rows(X, _lib.int8lt_quantize_rows_zp(dev(X)))
 
 
-def test_zp_prepare_weight_bit_exact():
-    w = wl.random_case(72, 4, 4096, 520)
+@pytest.mark.parametrize("N,K", [(520, 4096), (40, 144), (8, 16)])
+def test_zp_prepare_weight_bit_exact(N, K):
+    w = wl.random_case(72, 4, K, N)
     W = asymmetric_rows(wl.make_w(w))
-    check_zp_rows(W, _lib.int8lt_prepare_weight_zp(dev(W)))
+    CB, NDB, ZB, SB = _lib.int8lt_prepare_weight_zp(dev(W))
+    check_zp_rows(W, (_lib.int8lt_unpack_weight(CB, N, K), NDB, ZB, SB))
+    # padding of the blocked layout is zero codes
+    assert torch.equal(_lib.int8lt_pack_weight(_lib.int8lt_unpack_weight(CB, N, K)), CB)
 
 
 def test_zp_codes_span_the_range():
@@ -152,7 +156,7 @@ def test_zp_halves_equal_forward(M):
     ws = _lib.workspace(M, 264, 512, "cuda")
     Y2 = torch.empty_like(Y1)
     _lib.int8lt_forward_zp_quantize(X, 264, ws)
-    _lib.int8lt_forward_zp_matmul(M, CB, NDB, ZB, SB, b, Y2, ws)
+    _lib.int8lt_forward_zp_matmul(M, 512, CB, NDB, ZB, SB, b, Y2, ws)
     assert torch.equal(Y1, Y2)
 
 
