@@ -55,6 +55,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--out", default=None, help="also append the JSON line to this file")
+    p.add_argument("--no-fp16-weights", action="store_true",
+                   help="drop the fp16 weight: outlier-column weights come from CB * SCB / 127")
     p.add_argument("--quant", choices=["absmax", "zeropoint"], default="absmax",
                    help="absmax + outlier decomposition (LLM.int8()), or zeropoint on both sides")
     return p.parse_args()
@@ -165,7 +167,7 @@ class ClockSampler:
 
 # --------------------------------------------------------------- CPU oracle --
 
-def oracle_forward(w: wl.Workload, X, W, b, quant: str):
+def oracle_forward(w: wl.Workload, X, W, b, quant: str, keep_w: bool = True):
     """The oracle's forward of the chosen quantization, as a function of the row sample."""
     import oracle
 
@@ -173,17 +175,19 @@ def oracle_forward(w: wl.Workload, X, W, b, quant: str):
         CB, NDB, ZB, SB = oracle.zp_quantize_rows(W)
         return lambda rows: oracle.zp_forward(X, CB, NDB, ZB, SB, b, rows=rows)
     CB, SCB = oracle.prepare_weight(W)
-    return lambda rows: oracle.forward(X, CB, SCB, W, w.threshold, b, rows=rows)
+    Wo = W if keep_w else None
+    return lambda rows: oracle.forward(X, CB, SCB, Wo, w.threshold, b, rows=rows)
 
 
-def cpu_oracle_sample(w: wl.Workload, target_s: float, X=None, W=None, quant: str = "absmax"):
+def cpu_oracle_sample(w: wl.Workload, target_s: float, X=None, W=None, quant: str = "absmax",
+                      keep_w: bool = True):
     """Time the oracle forward on the first r rows of the workload (r sized to target_s)."""
     if X is None:
         X = wl.make_x(w)
     if W is None:
         W = wl.make_w(w)
     b = wl.make_bias(w)
-    fwd = oracle_forward(w, X, W, b, quant)   # weight conversion inside: offline, not timed
+    fwd = oracle_forward(w, X, W, b, quant, keep_w)   # weight conversion inside: offline, not timed
     probe = min(w.M, 8)
     t0 = time.perf_counter()
     fwd(np.arange(probe))
@@ -214,7 +218,7 @@ def run_reference(args, rank: int, world: int):
     w = wl.WORKLOADS[args.workload]
     X, W = wl.make_x(w), wl.make_w(w)
     b = wl.make_bias(w)
-    fwd = oracle_forward(w, X, W, b, args.quant)
+    fwd = oracle_forward(w, X, W, b, args.quant, not getattr(args, "no_fp16_weights", False))
     t0 = time.perf_counter()
     fwd(np.arange(1))
     t_row = time.perf_counter() - t0
@@ -290,6 +294,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     b = wl.make_bias(w)
     Xh = torch.from_numpy(X).pin_memory()
     Wd = torch.from_numpy(W).to(dev)
+    keep_w = not args.no_fp16_weights and args.quant == "absmax"
+    Wo = Wd if keep_w else None  # the fp16 weight the forward reads for the outlier columns
     bd = torch.from_numpy(b).to(dev) if b is not None else None
     zp = args.quant == "zeropoint"
     if zp:
@@ -303,19 +309,19 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if zp:
             _lib.int8lt_forward_zp(Xd, CB, NDB, ZB, SB, bd, Y, ws, st)
         else:
-            _lib.int8lt_forward(Xd, CB, SCB, Wd, w.threshold, bd, Y, ws, st)
+            _lib.int8lt_forward(Xd, CB, SCB, Wo, w.threshold, bd, Y, ws, st)
 
     def fwd_quantize(Xd, CB, ws, st):
         if zp:
             _lib.int8lt_forward_zp_quantize(Xd, N, ws, st)
         else:
-            _lib.int8lt_forward_quantize(Xd, CB, SCB, Wd, w.threshold, ws, st)
+            _lib.int8lt_forward_quantize(Xd, CB, SCB, Wo, w.threshold, ws, st)
 
     def fwd_matmul(CB, Y, ws, st):
         if zp:
             _lib.int8lt_forward_zp_matmul(M, K, CB, NDB, ZB, SB, bd, Y, ws, st)
         else:
-            _lib.int8lt_forward_matmul(M, K, CB, SCB, Wd, bd, Y, ws, st)
+            _lib.int8lt_forward_matmul(M, K, CB, SCB, Wo, bd, Y, ws, st)
 
     # Rotating input sets: X, CB, Y and workspace per set.
     ws_bytes = _lib.int8lt_workspace_size(M, N, K)
@@ -489,6 +495,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "parallelism": f"replicas x{world}", "quant": args.quant,
                    "cuda_graphs": f"up to {STEPS_PER_GRAPH} whole steps per graph, no event nodes inside"},
         "tokens_per_s": tokens_per_s,
+        "memory": {"layer_bytes": _lib.int8lt_weight_bytes(N, K) + (12 * N if zp else 4 * N)
+                   + (2 * N * K if keep_w else 0),
+                   "fp16_layer_bytes": 2 * N * K, "fp16_weight_kept": keep_w,
+                   "workspace_bytes": ws_bytes},
         "phases_ms": {"quantize": q_avg * 1e3, "matmul": m_avg * 1e3,
                       "how": "each half alone over the same steps, back to back from graphs"},
         "roofline": roof,
@@ -497,7 +507,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": sampler.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W, args.quant)
+        line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W, args.quant, keep_w)
     elif not args.no_cpu_baseline:
         line["cpu_baseline"] = None
     emit(line, args.out)

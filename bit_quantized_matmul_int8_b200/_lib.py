@@ -30,7 +30,7 @@ EXPORTS = [
     "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
     "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
     "int8lt_forward_zp_quantize", "int8lt_forward_zp_matmul",
-    "int8lt_weight_bytes", "int8lt_pack_weight", "int8lt_unpack_weight",
+    "int8lt_weight_bytes", "int8lt_pack_weight", "int8lt_unpack_weight", "int8lt_layer_bytes",
 ]
 
 
@@ -66,6 +66,7 @@ _SIGS = {
     "int8lt_forward_zp": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8lt_forward_zp_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _SZ, _P]),
     "int8lt_weight_bytes": (_SZ, [_I64, _I64]),
+    "int8lt_layer_bytes": (_SZ, [_I64, _I64, ctypes.c_int]),
     "int8lt_pack_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "int8lt_unpack_weight": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "int8lt_forward_zp_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -164,6 +165,11 @@ def _check_cb(CB: torch.Tensor, N: int, K: int) -> None:
 
 def int8lt_weight_bytes(N: int, K: int) -> int:
     return int(lib().int8lt_weight_bytes(N, K))
+
+
+def int8lt_layer_bytes(N: int, K: int, keep_fp16_weight: bool) -> int:
+    """Resident device bytes of a prepared [N,K] layer (CB + SCB [+ fp16 W])."""
+    return int(lib().int8lt_layer_bytes(N, K, int(bool(keep_fp16_weight))))
 
 
 def int8lt_pack_weight(CB_rows: torch.Tensor, stream=None) -> torch.Tensor:

@@ -228,6 +228,12 @@ size_t int8lt_weight_bytes(int64_t N, int64_t K) {
     return (size_t)weight_bytes(N, K);
 }
 
+size_t int8lt_layer_bytes(int64_t N, int64_t K, int keep_fp16_weight) {
+    const size_t w = int8lt_weight_bytes(N, K);
+    if (w == 0 && !(N == 0 && K >= 1)) return 0;
+    return w + 4 * (size_t)N + (keep_fp16_weight ? 2 * (size_t)N * (size_t)K : 0);
+}
+
 static int convert_weight(bool pack, const int8_t *src, int64_t N, int64_t K, int8_t *dst, void *stream) {
     if (N < 0 || K < 1 || K > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return INT8LT_ERR_SHAPE;
     if (N == 0) return INT8LT_OK;

@@ -125,6 +125,20 @@ int int8lt_pack_weight(const int8_t *CB_rows, int64_t N, int64_t K, int8_t *CB, 
 int int8lt_unpack_weight(const int8_t *CB, int64_t N, int64_t K, int8_t *CB_rows, void *stream);
 
 /*
+ * Memory accounting of a prepared layer: the device bytes it keeps resident
+ * between calls, CB (int8lt_weight_bytes(N, K)) + SCB (4 N), plus the fp16
+ * weight (2 N K) when the caller keeps it to serve the outlier columns
+ * (keep_fp16_weight != 0, W_outlier non-NULL). Against the 2 N K bytes of the
+ * fp16 layer this is about 50% without the fp16 weight, the saving the
+ * "LLM.int8() paper summary" states ("Int8 Matrix Multiplication at Scale");
+ * the outlier term then costs no extra weight memory, because its fp16
+ * weights are recovered from CB and SCB ([HF] has_fp16_weights=False). The
+ * per-call workspace (int8lt_workspace_size) is transient and not counted.
+ * Returns 0 for N < 0 or K < 1.
+ */
+size_t int8lt_layer_bytes(int64_t N, int64_t K, int keep_fp16_weight);
+
+/*
  * Weight conversion: W fp16 [N, K] -> CB int8 [N, K] (blocked weight
  * layout, int8lt_weight_bytes(N, K) bytes) and SCB fp32 [N].
  * [HF] "transformers integration": weights become int8 in [-127, 127] with a

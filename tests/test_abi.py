@@ -126,6 +126,22 @@ def test_zeropoint_entry_validation(L):
     assert m(32, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE + 8, FAKE, ws, None) == E["INT8LT_ERR_ALIGN"]
 
 
+def test_layer_memory_accounting(L):
+    # "LLM.int8() paper summary", "Int8 Matrix Multiplication at Scale": about
+    # half the memory of the fp16 layer once the fp16 weight is dropped.
+    for N, K in [(4096, 4096), (16384, 4096), (4096, 16384), (49152, 12288), (36864, 12288)]:
+        fp16 = 2 * N * K
+        b = L.int8lt_layer_bytes(N, K, 0)
+        assert b == L.int8lt_weight_bytes(N, K) + 4 * N == N * K + 4 * N
+        assert 0.5 <= b / fp16 <= 0.5 + 1e-3
+        assert L.int8lt_layer_bytes(N, K, 1) == b + fp16
+    # the blocked layout pads to 32 channels x 128 bytes
+    assert L.int8lt_weight_bytes(40, 136) == 2 * 2 * 4096
+    assert L.int8lt_layer_bytes(40, 136, 0) == 2 * 2 * 4096 + 160
+    assert L.int8lt_weight_bytes(-1, 16) == 0 and L.int8lt_weight_bytes(8, 0) == 0
+    assert L.int8lt_layer_bytes(-1, 16, 0) == 0 and L.int8lt_layer_bytes(8, 0, 1) == 0
+
+
 def test_product_path_does_not_touch_oracle():
     pkg = os.path.join(ROOT, "bit_quantized_matmul_int8_b200")
     for dirpath, _, files in os.walk(pkg):
