@@ -96,6 +96,30 @@ def test_quantize_rows_bit_exact(name, w, _, thr):
         assert host(idx).tolist() == wl.outlier_columns(w).tolist()
 
 
+@pytest.mark.parametrize("M,K", [(40, 256), (300, 1040), (2048, 4096), (17, 4096)])
+def test_quantize_row_max_in_other_rows_outlier_column(M, K):
+    """A row whose largest magnitude sits in a column that only other rows make an
+    outlier: its scale must come from the columns outside O (a ([P] decomposition)
+    case where a row cannot decide its own scale before the batch's O is known)."""
+    rng = np.random.default_rng(M + K)
+    X = np.clip(rng.standard_normal((M, K)) * 0.5, -2.5, 2.5).astype(np.float16)
+    X[0, 7] = 10.0                  # column 7 is an outlier column (row 0)
+    X[1, 7] = 5.5                   # row 1's max, below the threshold, in column 7
+    X[2, 7] = -5.9                  # row 2's max, negative
+    X[3, 7] = 3.0                   # row 3: its max is tied between column 7 and 20
+    X[3, 20] = 3.0
+    X[4, :] = 0.0
+    X[4, 7] = 1.0                   # row 4: its only non-zero is in O -> scale 0
+    X[5, K - 1] = 7.0               # another outlier column at the last position
+    X[6, K - 1] = -4.0
+    CA, SCA, idx = _lib.int8lt_quantize_rows(dev(X), 6.0)
+    CAo, SCAo, idxo = oracle.quantize_rows(X, 6.0)
+    assert host(idx).tolist() == idxo.tolist() == [7, K - 1]
+    assert np.array_equal(host(SCA).view(np.uint32), SCAo.view(np.uint32))
+    assert np.array_equal(host(CA), CAo)
+    assert host(SCA)[4] == 0.0 and float(host(SCA)[1]) < 5.5
+
+
 def test_quantize_threshold_boundary():
     X = np.zeros((40, 64), np.float16)
     X[3, 5] = 6.0
