@@ -55,6 +55,11 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--out", default=None, help="also append the JSON line to this file")
+    p.add_argument("--split", action="store_true",
+                   help="shard W by output channel over the ranks (strong scaling) instead of "
+                        "running a replica per rank")
+    p.add_argument("--gather", action="store_true",
+                   help="with --split: all-gather the Y shards every step (NCCL)")
     p.add_argument("--no-fp16-weights", action="store_true",
                    help="drop the fp16 weight: outlier-column weights come from CB * SCB / 127")
     p.add_argument("--quant", choices=["absmax", "zeropoint"], default="absmax",
@@ -287,11 +292,23 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     w = wl.WORKLOADS[args.workload]
     M, N, K = w.M, w.N, w.K
+    N_full = N
     peaks = load_peaks()
 
     X = wl.make_x(w)
     W = wl.make_w(w)
     b = wl.make_bias(w)
+    split = args.split and world > 1
+    if split:
+        # This rank's output channels; X is whole on every rank.
+        from bit_quantized_matmul_int8_b200.shard import gather_shards, shard_rows
+
+        n0, n1 = shard_rows(N, world, rank)
+        if n1 <= n0:
+            raise ValueError(f"--split: N={N} leaves rank {rank} of {world} no output channels")
+        W = np.ascontiguousarray(W[n0:n1])
+        b = np.ascontiguousarray(b[n0:n1]) if b is not None else None
+        N = n1 - n0
     Xh = torch.from_numpy(X).pin_memory()
     Wd = torch.from_numpy(W).to(dev)
     keep_w = not args.no_fp16_weights and args.quant == "absmax"
@@ -381,10 +398,21 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1)
 
-    graphs = graph_set()
-    for _ in range(max(1, math.ceil(max(3, args.warmup) / K_steps))):
-        for g in graphs:
+    gather = split and args.gather
+    if gather:
+        # One graph per step; the all-gather of the Y shards runs between them.
+        graphs = [capture(s0, s0 + 1) for s0 in range(K_steps)]
+    else:
+        graphs = graph_set()
+
+    def replay_steps():
+        for i, g in enumerate(graphs):
             g.replay()
+            if gather:
+                gather_shards(Ys[i % R], N_full)
+
+    for _ in range(max(1, math.ceil(max(3, args.warmup) / K_steps))):
+        replay_steps()
     torch.cuda.synchronize()
 
     dist = world > 1
@@ -398,8 +426,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     with sampler:
         t_start.record()
-        for g in graphs:
-            g.replay()
+        replay_steps()
         t_end.record()
         torch.cuda.synchronize()
     if dist:
@@ -421,9 +448,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if st != 0:
             raise RuntimeError(f"device status {_lib.STATUS.get(st)} after the timed steps")
 
-    ops = 2.0 * M * N * K
-    value = whole_job_rate(ops, K_steps, world, elapsed_ms) / 1e12
-    tokens_per_s = whole_job_rate(M, K_steps, world, elapsed_ms)
+    ops = 2.0 * M * N * K                     # this rank's matmul per step
+    if split:  # the ranks share one layer: the job does the whole layer per step
+        value = 2.0 * M * N_full * K * K_steps / (elapsed_ms * 1e-3) / 1e12
+        tokens_per_s = M * K_steps / (elapsed_ms * 1e-3)
+    else:
+        value = whole_job_rate(ops, K_steps, world, elapsed_ms) / 1e12
+        tokens_per_s = whole_job_rate(M, K_steps, world, elapsed_ms)
 
     # Roofline of the dominant kernel: the matmul half is one launch (GEMM or GEMV).
     src = ["bit_quantized_matmul_int8_b200/csrc/gemm_tc.cu" if not decode
@@ -478,21 +509,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-    e2e = {"value": whole_job_rate(ops, n_e2e, world, e2e_ms) / 1e12, "unit": "TOPS",
+    e2e_ops = 2.0 * M * N_full * K / world if split else ops  # per rank, whole job = x world
+    e2e = {"value": whole_job_rate(e2e_ops, n_e2e, world, e2e_ms) / 1e12, "unit": "TOPS",
            "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
-           "steps": n_e2e, "tokens_per_s": whole_job_rate(M, n_e2e, world, e2e_ms)}
+           "steps": n_e2e, "tokens_per_s": whole_job_rate(M, n_e2e, world, e2e_ms) / (world if split else 1)}
 
     if rank != 0:
         return
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K_steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": w.name, "M": M, "K": K, "N": N, "n_outliers": w.n_outliers,
+        "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": w.name, "M": M, "K": K, "N": N_full, "n_outliers": w.n_outliers,
                    "threshold": w.threshold, "x": "N(0,1) fp16 + planted outlier columns",
                    "w": f"N(0,{w.sigma_w}) fp16", "l2": f"{R} rotating input sets "
                    f"({R * touched / 2**20:.0f} MiB touched per cycle) > 126 MB L2",
-                   "parallelism": f"replicas x{world}", "quant": args.quant,
+                   "parallelism": (f"N split x{world} ({N} channels per rank"
+                                   + (", Y all-gathered" if gather else "") + ")") if split
+                   else f"replicas x{world}", "quant": args.quant,
                    "cuda_graphs": f"up to {STEPS_PER_GRAPH} whole steps per graph, no event nodes inside"},
         "tokens_per_s": tokens_per_s,
         "memory": {"layer_bytes": _lib.int8lt_weight_bytes(N, K) + (12 * N if zp else 4 * N)
