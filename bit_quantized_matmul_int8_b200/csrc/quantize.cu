@@ -186,6 +186,18 @@ __device__ __forceinline__ void flag_vec(uint4 x, uint32_t t2, int v, uint32_t *
     atomicOr(&bits[v >> 2], b << ((v & 3) * 8));
 }
 
+// Bit k set for the elements k of the vector whose magnitude bits equal m.
+__device__ __forceinline__ uint32_t elem_eq_mask(uint4 x, uint32_t m) {
+    const uint32_t w[4] = {x.x & 0x7fff7fffu, x.y & 0x7fff7fffu, x.z & 0x7fff7fffu, x.w & 0x7fff7fffu};
+    uint32_t b = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        b |= ((w[i] & 0xffffu) == m ? 1u : 0u) << (2 * i);
+        b |= ((w[i] >> 16) == m ? 1u : 0u) << (2 * i + 1);
+    }
+    return b;
+}
+
 // The vector with its outlier elements (bits of m) replaced by +0: their
 // code is then 0 and they do not count in the absmax.
 __device__ __forceinline__ uint4 clear_masked(uint4 x, uint32_t m) {
@@ -554,6 +566,258 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
         for (int64_t i = tid; i < a.cnt_words / 4; i += nth) reinterpret_cast<uint4 *>(a.cnt)[i] = make_uint4(0, 0, 0, 0);
 }
 
+// ------------------------------------------------ streaming, row per CTA --
+//
+// For batches with long rows (see launch_quantize) X is read from HBM once:
+// each CTA streams its rows, one row at a time across its 256 threads, with
+// the next row's loads in flight while the current one is quantized. A row's
+// elements with |x| >= threshold are outliers whatever the other rows hold,
+// so they are zeroed and the row's absmax and codes are taken over the rest
+// before the batch's outlier set O is known. After the grid barrier, with O
+// known, each row is finished: the columns of O it did not flag itself get
+// code 0 and their values go to Xo; the absmax stands unless every element
+// attaining it lies in O (the row's maximum falls in another row's outlier
+// column), in which case the row is quantized again from X with O masked.
+// Same results as quantize_kernel, bit for bit.
+constexpr int kStreamVpt = 8;                                  // 16-byte vectors per thread and row
+constexpr int64_t kStreamMaxK = (int64_t)kStreamVpt * kThreads * 8;  // 16384
+constexpr int kStreamMaxRows = 64;                             // rows per CTA
+constexpr int64_t kStreamMinK = 8192;                          // shorter rows: quantize_kernel
+
+// Outlier lanes of two fp16 values: bit 15 (low) / 31 (high) set where
+// |x| >= threshold. Exact integer arithmetic on the magnitude bits: 0x8000
+// above each 15-bit magnitude keeps the lanes' subtractions apart.
+__device__ __forceinline__ uint32_t ge_bits(uint32_t w, uint32_t t2) {
+    return (((w & 0x7fff7fffu) | 0x80008000u) - t2) & 0x80008000u;
+}
+
+// The 8 outlier flags of a vector as bits 0..7 (from ge_bits of its words).
+__device__ __forceinline__ uint32_t flags8(uint32_t g0, uint32_t g1, uint32_t g2, uint32_t g3) {
+    return ((g0 >> 15) & 1u) | ((g0 >> 30) & 2u) | ((g1 >> 13) & 4u) | ((g1 >> 28) & 8u) | ((g2 >> 11) & 16u) |
+           ((g2 >> 26) & 32u) | ((g3 >> 9) & 64u) | ((g3 >> 24) & 128u);
+}
+
+// Zero the flagged lanes of a word (g = its ge_bits).
+__device__ __forceinline__ uint32_t clear_flagged(uint32_t w, uint32_t g) { return w & ~((g >> 15) * 0xffffu); }
+
+__device__ __forceinline__ void stream_load(uint4 (&x)[kStreamVpt], const uint4 *row, int nvec, bool live) {
+#pragma unroll
+    for (int i = 0; i < kStreamVpt; ++i) {
+        const int v = threadIdx.x + kThreads * i;
+        x[i] = (live && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// Quantize one row held in x (one CTA): own outliers zeroed, absmax over the
+// rest, codes to CA. Records the absmax and a vector attaining it.
+__device__ __forceinline__ void stream_row(const QuantizeArgs &a, uint4 (&x)[kStreamVpt], int64_t r, int j, int nvec,
+                                           uint32_t t2, uint32_t *bits, uint32_t (*s_wmax)[kWarps],
+                                           int (*s_wv)[kWarps], uint32_t *s_amax, int32_t *s_vmax) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t mx = 0;
+    int mv = 0;
+#pragma unroll
+    for (int i = 0; i < kStreamVpt; ++i) {
+        const int v = threadIdx.x + kThreads * i;
+        if (v < nvec) {
+            const uint32_t g0 = ge_bits(x[i].x, t2), g1 = ge_bits(x[i].y, t2);
+            const uint32_t g2 = ge_bits(x[i].z, t2), g3 = ge_bits(x[i].w, t2);
+            if (g0 | g1 | g2 | g3) {
+                atomicOr(&bits[v >> 2], flags8(g0, g1, g2, g3) << ((v & 3) * 8));
+                x[i] = make_uint4(clear_flagged(x[i].x, g0), clear_flagged(x[i].y, g1), clear_flagged(x[i].z, g2),
+                                  clear_flagged(x[i].w, g3));
+            }
+            const uint32_t vm = vec_absmax_bits(x[i]);
+            if (vm > mx) {
+                mx = vm;
+                mv = v;
+            }
+        }
+    }
+    const uint32_t wm = warp_max_u32(mx);
+    const uint32_t who = __ballot_sync(0xffffffffu, mx == wm);
+    const int wv = __shfl_sync(0xffffffffu, mv, __ffs(who) - 1);
+    uint32_t(&cm)[kWarps] = s_wmax[j & 1];
+    int(&cv)[kWarps] = s_wv[j & 1];
+    if (lane == 0) {
+        cm[warp] = wm;
+        cv[warp] = wv;
+    }
+    __syncthreads();
+    uint32_t amax = cm[0];
+    int vmax = cv[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w)
+        if (cm[w] > amax) {
+            amax = cm[w];
+            vmax = cv[w];
+        }
+    const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+    const float sc = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+    uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+#pragma unroll
+    for (int i = 0; i < kStreamVpt; ++i) {
+        const int v = threadIdx.x + kThreads * i;
+        if (v < nvec) ca2[v] = quant_vec8(x[i], sc);
+    }
+    if (threadIdx.x == 0) {
+        s_amax[j] = amax;
+        s_vmax[j] = vmax;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) quantize_stream_kernel(QuantizeArgs a) {
+    extern __shared__ __align__(128) uint32_t smem[];
+    __shared__ uint32_t s_wmax[2][kWarps];
+    __shared__ int s_wv[2][kWarps];
+    __shared__ uint32_t s_amax[kStreamMaxRows];
+    __shared__ int32_t s_vmax[kStreamMaxRows];
+    __shared__ uint32_t s_gen, s_base;
+    const int64_t kwords = ceil_div(a.K, 32);
+    uint32_t *bits = smem;                                         // [kwords]
+    int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = (int)(a.K / 8);
+    const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
+    const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
+    const int nrows = a.M > blockIdx.x ? (int)ceil_div(a.M - blockIdx.x, gridDim.x) : 0;
+    grid_dep_launch();
+
+    uint4 xa[kStreamVpt], xb[kStreamVpt];
+    stream_load(xa, X4 + (int64_t)blockIdx.x * nvec, nvec, nrows > 0);
+    if (threadIdx.x == 0) {
+        s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
+        s_base = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qbase);
+    }
+    for (int64_t w = threadIdx.x; w < kwords; w += kThreads) bits[w] = 0;
+    __syncthreads();
+    const uint32_t gen = s_gen;
+    uint32_t *cur = a.bitmaps + (gen & 1u) * kMaxKwords;
+    uint32_t *nxt = a.bitmaps + ((gen + 1u) & 1u) * kMaxKwords;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
+        nxt[i] = 0;
+
+    // Rows blockIdx.x + j * gridDim.x, two at a time (xa, xb alternate).
+    for (int j = 0; j < nrows; j += 2) {
+        const int64_t r0 = blockIdx.x + (int64_t)j * gridDim.x, r1 = r0 + gridDim.x;
+        stream_load(xb, X4 + (j + 1 < nrows ? r1 : r0) * nvec, nvec, j + 1 < nrows);
+        stream_row(a, xa, r0, j, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax);
+        if (j + 1 < nrows) {
+            stream_load(xa, X4 + (j + 2 < nrows ? r1 + gridDim.x : r1) * nvec, nvec, j + 2 < nrows);
+            stream_row(a, xb, r1, j + 1, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax);
+        }
+    }
+    __syncthreads();
+
+    // CB into L2 for the GEMM (as quantize_kernel), then the batch's O.
+    if (a.Wo && a.CB && a.N * a.K <= kPrefetchMaxBytes && threadIdx.x < 32) {
+        const int64_t bytes = weight_bytes(a.N, a.K);
+        const int64_t slice = round_up(ceil_div(bytes, gridDim.x), 4096);
+        const int64_t b0 = (int64_t)blockIdx.x * slice, b1 = min(bytes, b0 + slice);
+        for (int64_t off = b0 + (int64_t)threadIdx.x * 4096; off < b1; off += 32 * 4096) {
+            const uint32_t n = (uint32_t)(b1 - off < 4096 ? b1 - off : 4096);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.CB + off), "r"(n) : "memory");
+        }
+    }
+    for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
+        if (bits[w]) atomicOr(&cur[w], bits[w]);
+    if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
+    for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
+        uint32_t v = __ldcg(&cur[w]);
+        if (w == kwords - 1 && (a.K & 31)) v &= (1u << (a.K & 31)) - 1u;
+        bits[w] = v;
+    }
+    __syncthreads();
+    const int32_t n_out = build_prefix(bits, prefix, kwords);
+    const int32_t n16 = (n_out + 15) & ~15;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0 && a.n_outliers) *a.n_outliers = n_out;
+        if (a.outlier_idx) {
+            for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
+                uint32_t v = bits[w];
+                int32_t rk = prefix[w];
+                while (v) {
+                    a.outlier_idx[rk++] = (int32_t)(w * 32 + __ffs(v) - 1);
+                    v &= v - 1;
+                }
+            }
+        }
+    }
+
+    // Finish each row (a warp per row).
+    for (int j = warp; j < nrows; j += kWarps) {
+        const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+        uint32_t amax = s_amax[j];
+        const int vmax = s_vmax[j];
+        uint32_t keep = 1;
+        if (lane == 0 && amax != 0u) {
+            const uint4 xv = __ldg(X4 + r * nvec + vmax);
+            const uint32_t own = flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2), ge_bits(xv.z, t2), ge_bits(xv.w, t2));
+            keep = (elem_eq_mask(xv, amax) & ~own & ~vec_mask(bits, vmax)) != 0u;
+        }
+        keep = __shfl_sync(0xffffffffu, keep, 0);
+        uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
+        if (!keep) {
+            // The row's maximum lies in O: absmax and codes again with O masked.
+            uint32_t m2 = 0;
+            for (int v = lane; v < nvec; v += 32) {
+                uint4 xv = __ldg(X4 + r * nvec + v);
+                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2),
+                                                              ge_bits(xv.z, t2), ge_bits(xv.w, t2));
+                m2 = max(m2, vec_absmax_bits(m ? clear_masked(xv, m) : xv));
+            }
+            amax = warp_max_u32(m2);
+            const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+            const float sc = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
+            for (int v = lane; v < nvec; v += 32) {
+                uint4 xv = __ldg(X4 + r * nvec + v);
+                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2),
+                                                              ge_bits(xv.z, t2), ge_bits(xv.w, t2));
+                ca2[v] = quant_vec8(m ? clear_masked(xv, m) : xv, sc);
+            }
+            __syncwarp();
+        }
+        // Columns of O: code 0 and the fp16 value into Xo (zero-padded to 16).
+        __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
+        const __half *xh = a.X + r * a.K;
+        for (int32_t t = lane; t < n16; t += 32) {
+            __half val = __float2half_rn(0.f);
+            if (t < n_out) {
+                const int64_t col = outlier_column(bits, prefix, kwords, t);
+                val = xh[col];
+                a.CA[r * a.K + col] = 0;
+            }
+            if (xo) xo[t] = val;
+        }
+        if (lane == 0) a.SCA[r] = __half2float(__ushort_as_half((unsigned short)amax));
+    }
+
+    // Outlier-weight gather Wo[j, t] (as quantize_kernel).
+    if (a.Wo && n16 > 0) {
+        const int hl = lane & 15;
+        const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
+        const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
+        const int64_t KB = wblocks_k(a.K);
+        for (int32_t t0 = 0; t0 < n16; t0 += 16) {
+            const int32_t t = t0 + hl;
+            const bool real = t < n_out;
+            const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
+            for (int64_t jj = hw; jj < a.N; jj += nhw) {
+                __half g = __float2half_rn(0.f);
+                if (real) {
+                    if (a.W_outlier) {
+                        g = a.W_outlier[jj * a.K + col];
+                    } else {
+                        const float p = __fmul_rn((float)a.CB[cb_offset(jj, col, KB)], a.SCB[jj]);
+                        g = __float2half_rn(__fdiv_rn(p, 127.f));
+                    }
+                }
+                a.Wo[jj * a.kcap + t] = g;
+            }
+        }
+    }
+}
+
 }  // namespace
 
 // --------------------------------------------------------------- host ----
@@ -626,7 +890,45 @@ cudaError_t quant_resident(int dyn, int *ctas) {
 
 }  // namespace
 
+// Resident CTAs of quantize_stream_kernel on the current device (cached;
+// its shared memory is at most 4 KB of bitmap and prefix, whatever K).
+cudaError_t stream_resident(int *ctas) {
+    static int cached[64];
+    static std::once_flag once[64];
+    static cudaError_t err[64];
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return e;
+    std::call_once(once[dev & 63], [dev] {
+        int sms = 0, per_sm = 0;
+        err[dev & 63] = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err[dev & 63] == cudaSuccess)
+            err[dev & 63] = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, quantize_stream_kernel, kThreads, (size_t)2 * (kStreamMaxK / 32) * 4);
+        cached[dev & 63] = sms * per_sm;
+    });
+    *ctas = cached[dev & 63];
+    return err[dev & 63];
+}
+
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
+    // Prefill batches with long rows: X streamed once, a row per CTA at a time.
+    if (a.M > kDecodeMaxM && a.K >= kStreamMinK && a.K <= kStreamMaxK && !a.acc && !a.cnt) {
+        int resident = 0;
+        if (cudaError_t e = stream_resident(&resident)) return e;
+        if (resident > 0 && ceil_div(a.M, resident) <= kStreamMaxRows) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+            cfg.gridDim = dim3((unsigned)std::min<int64_t>(resident, a.M), 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = (size_t)2 * ceil_div(a.K, 32) * 4;
+            cfg.stream = s;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            return cudaLaunchKernelEx(&cfg, quantize_stream_kernel, a);
+        }
+    }
     const int64_t kwords = ceil_div(a.K, 32);
     const int64_t bits_bytes = round_up(2 * kwords * 4, 128);
     const int64_t row_bytes = 2 * a.K;

@@ -77,6 +77,8 @@ QCASES = [
     ("rounds", wl.random_case(45, 4000, 4096, 8, n_outliers=7, frac=0.5), None),
     # rows of K >= 8192 are quantized by a whole CTA each, in rounds
     ("long_rows", wl.random_case(46, 1000, 16384, 8, n_outliers=4, frac=0.75), None),
+    # long rows, ragged vector count, a few rows per CTA (streamed, a row per CTA)
+    ("long_ragged", wl.random_case(48, 610, 10256, 8, n_outliers=5, frac=0.4), None),
     # rows too long to keep in shared memory: read from X in both phases
     ("very_long_rows", wl.random_case(47, 20, 65536, 8, n_outliers=3, frac=0.5), None),
 ]
@@ -96,7 +98,8 @@ def test_quantize_rows_bit_exact(name, w, _, thr):
         assert host(idx).tolist() == wl.outlier_columns(w).tolist()
 
 
-@pytest.mark.parametrize("M,K", [(40, 256), (300, 1040), (2048, 4096), (17, 4096)])
+@pytest.mark.parametrize("M,K", [(40, 256), (300, 1040), (2048, 4096), (17, 4096), (40, 8192), (33, 8208),
+                                 (300, 16384), (700, 12288)])
 def test_quantize_row_max_in_other_rows_outlier_column(M, K):
     """A row whose largest magnitude sits in a column that only other rows make an
     outlier: its scale must come from the columns outside O (a ([P] decomposition)
@@ -223,6 +226,7 @@ FCASES = [
     wl.random_case(57, 600, 2048, 1024, n_outliers=70, frac=0.2),  # > 64 outliers
     wl.random_case(58, 200, 384, 136, n_outliers=0),
     wl.random_case(63, 7, 3008, 20000, n_outliers=5, frac=1.0),   # decode, split row blocks
+    wl.random_case(64, 300, 12288, 264, n_outliers=9, frac=0.3),  # long rows, streamed quantize
 ]
 
 
