@@ -744,52 +744,99 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_stream_kernel(QuantizeAr
         }
     }
 
-    // Finish each row (a warp per row).
-    for (int j = warp; j < nrows; j += kWarps) {
-        const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
-        uint32_t amax = s_amax[j];
-        const int vmax = s_vmax[j];
-        uint32_t keep = 1;
-        if (lane == 0 && amax != 0u) {
-            const uint4 xv = __ldg(X4 + r * nvec + vmax);
+    // Finish the rows, a warp per row (rows warp, warp + 8, ...). Lane l first
+    // checks whether row warp + 8 l keeps its absmax: some element outside O
+    // attains it (else the row's maximum lies in O and the row is redone).
+    __shared__ int32_t s_redo[kStreamMaxRows];
+    __shared__ int32_t s_nredo;
+    if (threadIdx.x == 0) s_nredo = 0;
+    __syncthreads();
+    constexpr int kRowsPerWarp = kStreamMaxRows / kWarps;
+    uint32_t keep = 1;
+    {
+        const int j = warp + kWarps * lane;
+        if (lane < kRowsPerWarp && j < nrows && s_amax[j] != 0u) {
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            const uint4 xv = __ldg(X4 + r * nvec + s_vmax[j]);
             const uint32_t own = flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2), ge_bits(xv.z, t2), ge_bits(xv.w, t2));
-            keep = (elem_eq_mask(xv, amax) & ~own & ~vec_mask(bits, vmax)) != 0u;
+            keep = (elem_eq_mask(xv, s_amax[j]) & ~own & ~vec_mask(bits, s_vmax[j])) != 0u;
         }
-        keep = __shfl_sync(0xffffffffu, keep, 0);
+    }
+    const uint32_t keep_mask = __ballot_sync(0xffffffffu, keep);
+    // Columns of O: code 0 and the fp16 value into Xo (zero-padded to 16). With
+    // |O| <= 32 lane t owns rank t in every row, its loads issued together.
+    if (n16 <= 32) {
+        const int64_t col = lane < n_out ? outlier_column(bits, prefix, kwords, lane) : 0;
+        __half vals[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int j = warp + kWarps * i;
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            vals[i] = (j < nrows && lane < n_out) ? a.X[r * a.K + col] : __float2half_rn(0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int j = warp + kWarps * i;
+            if (j >= nrows) break;
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            if (lane < n_out) a.CA[r * a.K + col] = 0;
+            if (a.Xo && lane < n16) a.Xo[r * a.kcap + lane] = vals[i];
+        }
+    } else {
+        for (int j = warp; j < nrows; j += kWarps) {
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            for (int32_t t = lane; t < n16; t += 32) {
+                __half val = __float2half_rn(0.f);
+                if (t < n_out) {
+                    const int64_t col = outlier_column(bits, prefix, kwords, t);
+                    val = a.X[r * a.K + col];
+                    a.CA[r * a.K + col] = 0;
+                }
+                if (a.Xo) a.Xo[r * a.kcap + t] = val;
+            }
+        }
+    }
+    for (int i = 0, j = warp; j < nrows; ++i, j += kWarps) {
+        if ((keep_mask >> i) & 1u) {
+            if (lane == 0) a.SCA[blockIdx.x + (int64_t)j * gridDim.x] = __half2float(__ushort_as_half((unsigned short)s_amax[j]));
+        } else if (lane == 0) {
+            s_redo[atomicAdd(&s_nredo, 1)] = j;
+        }
+    }
+    __syncthreads();
+    // Rows whose maximum lies in O: the whole CTA quantizes them again from X
+    // with O masked (rare: a row's maximum in another row's outlier column).
+    const int nredo = s_nredo;
+    for (int k = 0; k < nredo; ++k) {
+        const int j = s_redo[k];
+        const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+        stream_load(xa, X4 + r * nvec, nvec, true);
+        uint32_t mx = 0;
+#pragma unroll
+        for (int i = 0; i < kStreamVpt; ++i) {
+            const int v = threadIdx.x + kThreads * i;
+            if (v < nvec) {
+                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xa[i].x, t2), ge_bits(xa[i].y, t2),
+                                                              ge_bits(xa[i].z, t2), ge_bits(xa[i].w, t2));
+                if (m) xa[i] = clear_masked(xa[i], m);
+                mx = max(mx, vec_absmax_bits(xa[i]));
+            }
+        }
+        mx = warp_max_u32(mx);
+        if (lane == 0) s_wmax[k & 1][warp] = mx;
+        __syncthreads();
+        uint32_t amax = s_wmax[k & 1][0];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) amax = max(amax, s_wmax[k & 1][w]);
+        const float sa = __half2float(__ushort_as_half((unsigned short)amax));
+        const float sc = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
         uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
-        if (!keep) {
-            // The row's maximum lies in O: absmax and codes again with O masked.
-            uint32_t m2 = 0;
-            for (int v = lane; v < nvec; v += 32) {
-                uint4 xv = __ldg(X4 + r * nvec + v);
-                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2),
-                                                              ge_bits(xv.z, t2), ge_bits(xv.w, t2));
-                m2 = max(m2, vec_absmax_bits(m ? clear_masked(xv, m) : xv));
-            }
-            amax = warp_max_u32(m2);
-            const float sa = __half2float(__ushort_as_half((unsigned short)amax));
-            const float sc = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
-            for (int v = lane; v < nvec; v += 32) {
-                uint4 xv = __ldg(X4 + r * nvec + v);
-                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2),
-                                                              ge_bits(xv.z, t2), ge_bits(xv.w, t2));
-                ca2[v] = quant_vec8(m ? clear_masked(xv, m) : xv, sc);
-            }
-            __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kStreamVpt; ++i) {
+            const int v = threadIdx.x + kThreads * i;
+            if (v < nvec) ca2[v] = quant_vec8(xa[i], sc);
         }
-        // Columns of O: code 0 and the fp16 value into Xo (zero-padded to 16).
-        __half *xo = a.Xo ? a.Xo + r * a.kcap : nullptr;
-        const __half *xh = a.X + r * a.K;
-        for (int32_t t = lane; t < n16; t += 32) {
-            __half val = __float2half_rn(0.f);
-            if (t < n_out) {
-                const int64_t col = outlier_column(bits, prefix, kwords, t);
-                val = xh[col];
-                a.CA[r * a.K + col] = 0;
-            }
-            if (xo) xo[t] = val;
-        }
-        if (lane == 0) a.SCA[r] = __half2float(__ushort_as_half((unsigned short)amax));
+        if (threadIdx.x == 0) a.SCA[r] = sa;
     }
 
     // Outlier-weight gather Wo[j, t] (as quantize_kernel).
