@@ -569,8 +569,8 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
 // ------------------------------------------------ streaming, row per CTA --
 //
 // For batches with long rows (see launch_quantize) X is read from HBM once:
-// each CTA streams its rows, one row at a time across its 256 threads, with
-// the next row's loads in flight while the current one is quantized. A row's
+// each CTA streams its rows, one row at a time across its 256 threads (three
+// CTAs per SM, so one CTA's loads are in flight while the others quantize). A row's
 // elements with |x| >= threshold are outliers whatever the other rows hold,
 // so they are zeroed and the row's absmax and codes are taken over the rest
 // before the batch's outlier set O is known. After the grid barrier, with O
@@ -666,7 +666,7 @@ __device__ __forceinline__ void stream_row(const QuantizeArgs &a, uint4 (&x)[kSt
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) quantize_stream_kernel(QuantizeArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeArgs a) {
     extern __shared__ __align__(128) uint32_t smem[];
     __shared__ uint32_t s_wmax[2][kWarps];
     __shared__ int s_wv[2][kWarps];
@@ -683,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_stream_kernel(QuantizeAr
     const int nrows = a.M > blockIdx.x ? (int)ceil_div(a.M - blockIdx.x, gridDim.x) : 0;
     grid_dep_launch();
 
-    uint4 xa[kStreamVpt], xb[kStreamVpt];
+    uint4 xa[kStreamVpt];
     stream_load(xa, X4 + (int64_t)blockIdx.x * nvec, nvec, nrows > 0);
     if (threadIdx.x == 0) {
         s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
@@ -697,15 +697,11 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_stream_kernel(QuantizeAr
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
         nxt[i] = 0;
 
-    // Rows blockIdx.x + j * gridDim.x, two at a time (xa, xb alternate).
-    for (int j = 0; j < nrows; j += 2) {
-        const int64_t r0 = blockIdx.x + (int64_t)j * gridDim.x, r1 = r0 + gridDim.x;
-        stream_load(xb, X4 + (j + 1 < nrows ? r1 : r0) * nvec, nvec, j + 1 < nrows);
+    // Rows blockIdx.x + j * gridDim.x, one at a time.
+    for (int j = 0; j < nrows; ++j) {
+        const int64_t r0 = blockIdx.x + (int64_t)j * gridDim.x;
+        if (j > 0) stream_load(xa, X4 + r0 * nvec, nvec, true);
         stream_row(a, xa, r0, j, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax);
-        if (j + 1 < nrows) {
-            stream_load(xa, X4 + (j + 2 < nrows ? r1 + gridDim.x : r1) * nvec, nvec, j + 2 < nrows);
-            stream_row(a, xb, r1, j + 1, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax);
-        }
     }
     __syncthreads();
 
