@@ -8,10 +8,13 @@
 // Kernels (HBM-bound streaming passes):
 //   prepare_weight_kernel  W [N,K] -> CB, SCB          (one warp per row)
 //   quantize_kernel        one cooperative launch: the CTA's rows of X are
-//                          staged in shared memory by bulk copies; phase A
-//                          ORs the outlier columns of every row into a
-//                          bitmap, a grid barrier, then phase B writes O, CA,
-//                          SCA, Xo from the staged rows and gathers Wo
+//                          staged in shared memory; phase A ORs the outlier
+//                          columns of every row into a bitmap, a grid
+//                          barrier, then phase B writes O, CA, SCA, Xo from
+//                          the staged rows and gathers Wo
+//   quantize_stream_kernel prefill rows of 8192..16384 columns: X streamed
+//                          once, each row quantized with its own outliers
+//                          masked before the barrier and finished after it
 //
 // Exactness: |x| >= threshold is decided on the fp16 bit pattern against the
 // smallest fp16 pattern whose value reaches the fp32 threshold (the map from
