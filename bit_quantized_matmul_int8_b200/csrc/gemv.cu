@@ -11,8 +11,9 @@
 //   - warp w streams blocks [w L, (w + 1) L) of that sequence: one contiguous
 //     range per warp, the same length for every warp (balanced to one block
 //     over the whole grid, 3 CTAs of 8 warps per SM);
-//   - each lane issues 16-byte loads (8 per block, the block's 32 rows x 128
-//     bytes over the warp) and the matching CA bytes; mma.sync m16n8k32
+//   - each lane issues 256-bit loads (4 per block, the block's 32 rows x 128
+//     bytes over the warp; 16-byte loads when CB is only 16-byte aligned) and
+//     the matching CA bytes; mma.sync m16n8k32
 //     (int8 -> int32) with the tokens as the 16-row A operand and 8 weight
 //     rows as B. The K order inside one MMA is irrelevant to an exact integer
 //     sum, so the 16 bytes a lane loaded are used as they lie, with the same
@@ -45,6 +46,14 @@ __device__ __forceinline__ void mma_16832_s8(int32_t (&d)[4], const uint32_t (&a
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 32 contiguous bytes (one 256-bit load; p 32-byte aligned), read once:
+// not kept in L1 and first out of L2, so that CA stays cached.
+__device__ __forceinline__ void ld_stream32(const int8_t *p, uint4 &lo, uint4 &hi) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
 }
 
 __device__ __forceinline__ uint4 ld_stream(const int8_t *p) {
@@ -139,7 +148,9 @@ __device__ __forceinline__ void row_block_out(const GemvArgs &a, int n_out, int6
 // kHi: more than 8 tokens (the MMA's rows 8..15 are live). kOut: the
 // absmax forward, whose outlier term is read from the workspace (|O| may still
 // be 0); without it (zeropoint, raw int32 sums) no outlier code is compiled.
-template <bool kHi, bool kOut>
+// kWide: CB is 32-byte aligned, and each lane reads its 32 bytes of a block
+// row with one 256-bit load (else two 16-byte loads 64 bytes apart).
+template <bool kHi, bool kOut, bool kWide>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm)
 gemv_i8_kernel(const GemvArgs a, const int64_t L) {
     __shared__ float s_p[kOut ? kWarpsPerCta : 1][16][32];  // outlier products of a row block, per warp
@@ -169,7 +180,7 @@ gemv_i8_kernel(const GemvArgs a, const int64_t L) {
     const int n_out = kOut ? *a.n_outliers : 0;
     const uint4 z = make_uint4(0, 0, 0, 0);
     // This lane's 16-byte pieces of a block: rows 8q + g, bytes 64h + 16tig.
-    const int lane_off = g * kWBlockCols + tig * 16;
+    const int lane_off = g * kWBlockCols + tig * (kWide ? 32 : 16);
 
     while (s < s1) {
         const int64_t rb = s / KB;                      // row block
@@ -181,13 +192,20 @@ gemv_i8_kernel(const GemvArgs a, const int64_t L) {
             const int8_t *blk = a.CB + st * kWBlockBytes + lane_off;
             const int64_t kb = (st - rb * KB) * kWBlockCols;
             uint4 wv[2][4], xl[2], xh[2] = {z, z};
+            if constexpr (kWide) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ld_stream32(blk + q * 8 * kWBlockCols, wv[0][q], wv[1][q]);
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                // CB's padding columns are zero codes; CA stops at K.
-                const int64_t kk = kb + h * 64 + tig * 16;
+                // CB's padding columns are zero codes; CA stops at K. Piece h of
+                // this lane holds the same K positions of A and of B.
+                const int64_t kk = kb + (kWide ? tig * 32 + h * 16 : h * 64 + tig * 16);
                 const bool kin = kk < a.K;
+                if constexpr (!kWide) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) wv[h][q] = ld_stream(blk + q * 8 * kWBlockCols + h * 64);
+                    for (int q = 0; q < 4; ++q) wv[h][q] = ld_stream(blk + q * 8 * kWBlockCols + h * 64);
+                }
                 xl[h] = (kin && tok_lo) ? __ldg(reinterpret_cast<const uint4 *>(xa + kk)) : z;
                 if constexpr (kHi) xh[h] = (kin && tok_hi) ? __ldg(reinterpret_cast<const uint4 *>(xb + kk)) : z;
             }
@@ -246,7 +264,7 @@ cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s) {
         int sms = 0, per_sm = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_i8_kernel<true, true>,
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_i8_kernel<true, true, true>,
                                                               kWarpsPerCta * 32, 0);
         if (e != cudaSuccess) return e;
         resident[dev & 63] = std::max(1, sms * per_sm);
@@ -265,11 +283,19 @@ cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const bool out = a.n_outliers && !a.ZB && !a.C32;
+    const bool wide = (reinterpret_cast<uintptr_t>(a.CB) & 31) == 0;
+    if (wide) {
+        if (a.M > 8)
+            return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, true, true>, a, L)
+                       : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, false, true>, a, L);
+        return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, true, true>, a, L)
+                   : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, false, true>, a, L);
+    }
     if (a.M > 8)
-        return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, true>, a, L)
-                   : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, false>, a, L);
-    return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, true>, a, L)
-               : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, false>, a, L);
+        return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, true, false>, a, L)
+                   : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<true, false, false>, a, L);
+    return out ? cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, true, false>, a, L)
+               : cudaLaunchKernelEx(&cfg, gemv_i8_kernel<false, false, false>, a, L);
 }
 
 }  // namespace int8lt

@@ -204,6 +204,32 @@ def test_gemm_int32_matches_oracle_routine():
     assert np.array_equal(host(gemm_i32_gpu(A, B)), oracle.gemm_i32(A, B))
 
 
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_cb_only_16_byte_aligned(M):
+    """CB at an address that is 16- but not 32-byte aligned (the API's minimum): the
+    decode GEMV then reads it with 16-byte loads; results equal the aligned case."""
+    N, K = 264, 1040
+    rng = np.random.default_rng(M)
+    A = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    B = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    CB = _lib.int8lt_pack_weight(dev(B))
+    buf = torch.empty(CB.numel() + 32, dtype=torch.int8, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    CB16 = buf[16:16 + CB.numel()]
+    CB16.copy_(CB.view(-1))
+    assert CB16.data_ptr() % 32 == 16
+    C = host(_lib.int8lt_debug_gemm_i32(dev(A), CB16, N))
+    assert np.array_equal(C, oracle.gemm_i32(A, B))
+    w = wl.random_case(65, M, K, N, n_outliers=3, frac=1.0)
+    X, W, b = case_inputs(w)
+    CBw, SCB = _lib.int8lt_prepare_weight(dev(W))
+    CBw16 = buf[16:16 + CBw.numel()]
+    CBw16.copy_(CBw.view(-1))
+    Y1 = _lib.int8lt_forward(dev(X), CBw, SCB, dev(W), 6.0, dev(b))
+    Y2 = _lib.int8lt_forward(dev(X), CBw16, SCB, dev(W), 6.0, dev(b))
+    assert torch.equal(Y1, Y2)
+
+
 def test_gemm_int32_extreme_k():
     # K near the int32 limit: 127 * 127 * K stays below 2^31
     K = 133136
