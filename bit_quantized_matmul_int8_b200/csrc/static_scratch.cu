@@ -1,7 +1,7 @@
 // Allocation-free forward for decode shapes (M <= 16 tokens).
 //
 // int8lt_forward takes its scratch (outlier bitmap and list, CA/SCA, the
-// fp16 outlier activations, split-K partial sums) from a caller-provided
+// fp16 outlier activations, the GEMV's partial sums) from a caller-provided
 // workspace. Some callers cannot provide one: a plugin or engine that hands
 // this layer only its input and output buffers, a runtime whose device
 // memory is owned entirely by its own pool, or a latency-critical decode
@@ -13,7 +13,7 @@
 // The array is kStaticScratchBytes (8 MiB). Every GPU on which the library
 // is loaded holds it until the process exits. It is shared by all calls on
 // that GPU and keeps the previous call's contents: the quantize pass of every
-// call rewrites the outlier list, codes and scales and zeroes the split-K
+// call rewrites the outlier list, codes and scales and zeroes the GEMV's
 // sums before they are accumulated, so nothing carries over; but two calls
 // whose kernels overlap on the GPU (different streams without ordering, or
 // different host threads) race on the array and corrupt each other.

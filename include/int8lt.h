@@ -84,7 +84,8 @@ int int8lt_version(void);
  * Workspace bytes that int8lt_forward needs for an [M, K] x [N, K]^T call.
  * Holds the outlier bitmap partials, the outlier list and count, the device
  * status word, CA/SCA, the gathered fp16 outlier activations, and either the
- * gathered fp16 outlier weights (M > 16) or split-K int32 partials (M <= 16).
+ * gathered fp16 outlier weights (M > 16) or the decode GEMV's int32 partial
+ * sums of row blocks shared between warps (M <= 16).
  * The outlier buffers are sized for the worst case |O| = K, so any input fits.
  * Returns 0 for shapes the library rejects.
  */
@@ -180,7 +181,7 @@ int int8lt_quantize_rows(const void *X, int64_t M, int64_t K, float threshold,
  *               in O are read), or NULL to use fp16(fp32(CB * SCB) / 127).
  *   bias      : fp16 [N] or NULL.
  *   ws        : at least int8lt_workspace_size(M, N, K) bytes.
- * Dispatch: M <= 16 runs the memory-bound split-K GEMV; larger M runs the
+ * Dispatch: M <= 16 runs the memory-bound streaming GEMV; larger M runs the
  * tcgen05 int8 GEMM with the outlier MMA and the dequantization fused into it.
  */
 int int8lt_forward(const void *X, int64_t M, int64_t N, int64_t K,
