@@ -16,7 +16,7 @@
 //     the matching CA bytes; mma.sync m16n8k32
 //     (int8 -> int32) with the tokens as the 16-row A operand and 8 weight
 //     rows as B. The K order inside one MMA is irrelevant to an exact integer
-//     sum, so the 16 bytes a lane loaded are used as they lie, with the same
+//     sum, so the bytes a lane loaded are used as they lie, with the same
 //     permutation applied to A and B;
 //   - where a warp's range starts or ends inside a row block, its int32
 //     partial sums are added with atomics (exact in any order) and the last
@@ -25,8 +25,10 @@
 //   - launched with programmatic stream serialization, each warp pulls the
 //     first blocks of its range into L2 before it waits for the quantize pass.
 // A read-bandwidth probe on this machine measured this pattern at 6.1-6.4 TB/s
-// against 4.5 TB/s for 32 row-major rows read 128 bytes at a time, and
-// 5.1-5.3 TB/s for blocked rows split by row block alone (uneven per SM).
+// with 16-byte loads, against 4.5 TB/s for 32 row-major rows read 128 bytes
+// at a time and 5.1-5.3 TB/s for blocked rows split by row block alone
+// (uneven per SM); the 256-bit evict-first loads took the kernel to about
+// 6.3-6.8 TB/s.
 #include <algorithm>
 
 #include "int8lt_internal.cuh"
