@@ -142,6 +142,21 @@ def test_layer_memory_accounting(L):
     assert L.int8lt_layer_bytes(-1, 16, 0) == 0 and L.int8lt_layer_bytes(8, 0, 1) == 0
 
 
+def test_weight_layout_entry_validation(L):
+    E = _lib.STATUS_CODE
+    assert L.int8lt_weight_bytes(1, 1) == 4096 and L.int8lt_weight_bytes(33, 129) == 4 * 4096
+    assert L.int8lt_weight_bytes(0, 16) == 0
+    p, u = L.int8lt_pack_weight, L.int8lt_unpack_weight
+    assert p(None, 8, 16, FAKE, None) == E["INT8LT_ERR_NULL"]
+    assert p(FAKE, 8, 16, None, None) == E["INT8LT_ERR_NULL"]
+    assert p(FAKE, 8, 0, FAKE, None) == E["INT8LT_ERR_SHAPE"]
+    assert p(FAKE, -1, 16, FAKE, None) == E["INT8LT_ERR_SHAPE"]
+    assert p(FAKE, 8, 16, FAKE + 8, None) == E["INT8LT_ERR_ALIGN"]      # blocked codes: 16 bytes
+    assert p(FAKE + 8, 8, 16, FAKE, None) == E["INT8LT_ERR_ALIGN"]      # rows, K % 16 == 0: 16 bytes
+    assert u(FAKE + 8, 8, 16, FAKE, None) == E["INT8LT_ERR_ALIGN"]
+    assert p(None, 0, 16, None, None) == E["INT8LT_OK"]                 # empty: no-op
+
+
 def test_product_path_does_not_touch_oracle():
     pkg = os.path.join(ROOT, "bit_quantized_matmul_int8_b200")
     for dirpath, _, files in os.walk(pkg):
