@@ -30,6 +30,7 @@
 // (uneven per SM); the 256-bit evict-first loads took the kernel to about
 // 6.3-6.8 TB/s.
 #include <algorithm>
+#include <atomic>
 
 #include "int8lt_internal.cuh"
 
@@ -258,21 +259,25 @@ gemv_i8_kernel(const GemvArgs a, const int64_t L) {
 }  // namespace
 
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s) {
-    static int resident[64];  // CTAs of this kernel that fit on the device at once
+    // CTAs of this kernel that fit on the device at once (0: not known yet;
+    // threads that race on the first call compute and store the same value).
+    static std::atomic<int> resident[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (resident[dev & 63] == 0) {
+    int ctas = resident[dev & 63].load(std::memory_order_relaxed);
+    if (ctas == 0) {
         int sms = 0, per_sm = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e == cudaSuccess)
             e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_i8_kernel<true, true, true>,
                                                               kWarpsPerCta * 32, 0);
         if (e != cudaSuccess) return e;
-        resident[dev & 63] = std::max(1, sms * per_sm);
+        ctas = std::max(1, sms * per_sm);
+        resident[dev & 63].store(ctas, std::memory_order_relaxed);
     }
     const int64_t total = ceil_div(a.N, kWBlockRows) * wblocks_k(a.K);
-    const int64_t warps_max = (int64_t)resident[dev & 63] * kWarpsPerCta;
+    const int64_t warps_max = (int64_t)ctas * kWarpsPerCta;
     const int64_t L = std::max(kMinBlocksPerWarp, ceil_div(total, warps_max));
     const int64_t warps = ceil_div(total, L);
     cudaLaunchConfig_t cfg = {};
