@@ -97,3 +97,16 @@ def test_reference_arm_zeropoint(capsys):
     line = json.loads(capsys.readouterr().out.strip())
     assert line["impl"] == "reference" and line["config"]["quant"] == "zeropoint"
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_cpu_baseline_legs_all_modes():
+    """bench.py's CPU-baseline leg for each quantization and weight mode."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from bit_quantized_matmul_int8_b200 import workloads as wl
+
+    w = wl.WORKLOADS["tiny_16x64x64"]
+    for quant, keep_w in (("absmax", True), ("absmax", False), ("zeropoint", False)):
+        cb = bench.cpu_oracle_sample(w, 0.05, quant=quant, keep_w=keep_w)
+        assert cb["kind"] == "oracle" and cb["value"] > 0 and 1 <= cb["rows"] <= w.M
+        assert ("zeropoint" in cb["sample"]) == (quant == "zeropoint")
