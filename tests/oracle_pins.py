@@ -356,9 +356,26 @@ def pin_zp_forward_within_bound(lib):
     assert (np.abs(Y - ref) <= bound * (1 + 1e-6) + 1e-12).all()
 
 
+def pin_zp_worked_examples(lib):
+    """[HF] zero-point maps a range such as [-1, 1] onto [-127, 127]; [P4] nd and the
+    zeropoint shift: four rows worked by hand (``tests/golden/zeropoint_worked_examples.txt``),
+    including two ties that round to even."""
+    with open(os.path.join(GOLDEN, "zeropoint_worked_examples.txt")) as f:
+        rows = [ln.strip() for ln in f if ln.strip().startswith("row ")]
+    assert len(rows) == 4
+    for ln in rows:
+        parts = [p.split() for p in ln[4:].split("|")]
+        vals = np.array([float(v) for v in parts[0]], dtype=np.float16)[None, :]
+        nd, zp, codes = float(parts[1][1]), int(parts[2][1]), [int(c) for c in parts[3][1:]]
+        Q, ND, ZP, SUM = oracle.zp_quantize_rows(vals, lib=lib)
+        assert Q[0].tolist() == codes, (ln, Q[0].tolist())
+        assert int(ZP[0]) == zp and abs(float(ND[0]) - nd) <= 1e-5 * nd, ln
+        assert int(SUM[0]) == sum(codes)
+
+
 PINS = [pin_half_decode, pin_half_encode, pin_worked_example, pin_absmax_invariants,
         pin_weight_recovery, pin_outlier_bruteforce, pin_outlier_boundary,
         pin_planted_outliers, pin_row_scale_excludes_outliers, pin_round_ties_to_even, pin_gemm_exact,
         pin_gemm_overflow, pin_all_columns_outlier, pin_all_columns_outlier_int8_weights,
         pin_outlier_weight_gather, pin_forward_within_bound, pin_zp_invariants, pin_zp_unrolled_product,
-        pin_zp_forward_within_bound]
+        pin_zp_forward_within_bound, pin_zp_worked_examples]

@@ -37,6 +37,7 @@ MUTANTS = [
     ("half_encode_ties_away", "double r = nearbyint(ldexp(a, 10 - E));", "double r = round(ldexp(a, 10 - E));"),
     ("zp_drop_k_term", "+ K * (int64_t)za * ZPB[j];", ";"),
     ("zp_sign", "int64_t c = (int64_t)nearbyintf(h2f(x[h]) * nd) - z;", "int64_t c = (int64_t)nearbyintf(h2f(x[h]) * nd) + z;"),
+    ("zp_ties_away", "int64_t c = (int64_t)nearbyintf(h2f(x[h]) * nd) - z;", "int64_t c = (int64_t)roundf(h2f(x[h]) * nd) - z;"),
     ("zp_range_255", "float nd = range > 0.0f ? 254.0f / range : 1.0f;", "float nd = range > 0.0f ? 255.0f / range : 1.0f;"),
     ("zp_no_shift", "int32_t z = (int32_t)zmin + 127;", "int32_t z = (int32_t)zmin;"),
     ("zp_correction_swapped", "(int64_t)ZPB[j] * sa + (int64_t)za * SUMB[j]", "(int64_t)za * sa + (int64_t)ZPB[j] * SUMB[j]"),
