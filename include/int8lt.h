@@ -47,7 +47,9 @@
  *     and K % 16 == 0 (int8 rows must be 16-byte multiples for the TMA
  *     engine; 133144 * 127^2 < 2^31 keeps every int32 sum exact), N % 8 == 0.
  *   - Alignment: X, W, W_outlier, CB, CA, Y and the workspace must be 16-byte
- *     aligned; scale arrays 4-byte, bias 2-byte.
+ *     aligned; scale arrays 4-byte, bias 2-byte. A 32-byte aligned CB (any
+ *     cudaMalloc'd buffer is) lets the decode GEMV read it with 256-bit loads;
+ *     a CB that is only 16-byte aligned gives the same results, more slowly.
  *   - NaN or infinite values inside X or W are outside the contract.
  */
 #ifndef INT8LT_H
