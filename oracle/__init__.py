@@ -62,9 +62,6 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_outlier_columns.argtypes = [_P, _I64, _I64, ctypes.c_float, _P]
     lib.oracle_quantize_rows.restype = _I64
     lib.oracle_quantize_rows.argtypes = [_P, _I64, _I64, ctypes.c_float, _P, _P, _P]
-    lib.oracle_quantize_some_rows.restype = _I64
-    lib.oracle_quantize_some_rows.argtypes = [_P, _I64, _I64, ctypes.c_float, _P, _I64,
-                                              _P, _P, _P]
     lib.oracle_prepare_weight.restype = None
     lib.oracle_prepare_weight.argtypes = [_P, _I64, _I64, _P, _P]
     lib.oracle_gemm_i32.restype = ctypes.c_int
@@ -125,20 +122,6 @@ def quantize_rows(X: np.ndarray, threshold: float, lib=None):
     SCA = np.zeros(M, dtype=np.float32)
     idx = np.zeros(max(K, 1), dtype=np.int32)
     n = lib.oracle_quantize_rows(_ptr(x), M, K, float(threshold), _ptr(CA), _ptr(SCA), _ptr(idx))
-    return CA, SCA, idx[:n].copy()
-
-
-def quantize_some_rows(X: np.ndarray, threshold: float, rows, lib=None):
-    """Rows ``rows`` of quantize_rows (O still taken over all of X)."""
-    lib = lib or load()
-    x = _h(X)
-    M, K = x.shape
-    rows = np.ascontiguousarray(rows, dtype=np.int64)
-    CA = np.zeros((len(rows), K), dtype=np.int8)
-    SCA = np.zeros(len(rows), dtype=np.float32)
-    idx = np.zeros(max(K, 1), dtype=np.int32)
-    n = lib.oracle_quantize_some_rows(_ptr(x), M, K, float(threshold), _ptr(rows), len(rows),
-                                      _ptr(CA), _ptr(SCA), _ptr(idx))
     return CA, SCA, idx[:n].copy()
 
 

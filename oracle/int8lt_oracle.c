@@ -153,20 +153,6 @@ int64_t oracle_quantize_rows(const uint16_t *X, int64_t M, int64_t K, float thre
     return n_out;
 }
 
-/* Quantize only the listed rows of X (O is still taken over all rows). */
-int64_t oracle_quantize_some_rows(const uint16_t *X, int64_t M, int64_t K, float threshold,
-                                  const int64_t *rows, int64_t nrows,
-                                  int8_t *CA, float *SCA, int32_t *outlier_idx)
-{
-    int64_t n_out = oracle_outlier_columns(X, M, K, threshold, outlier_idx);
-    unsigned char *mask = (unsigned char *)calloc((size_t)K, 1);
-    for (int64_t t = 0; t < n_out; ++t) mask[outlier_idx[t]] = 1;
-    for (int64_t r = 0; r < nrows; ++r)
-        SCA[r] = quantize_vector(X + rows[r] * K, mask, K, CA + r * K);
-    free(mask);
-    return n_out;
-}
-
 /* [P2 transformers integration]: weights W [N, K] become int8 CB in
  * [-127, 127] with one scale SCB_j per output channel j (absmax over all K),
  * so that W ~= CB * SCB / 127. */

@@ -280,6 +280,35 @@ def pin_forward_within_bound(lib):
             assert np.array_equal(Y16, Y64.astype(np.float16))
 
 
+def pin_row_subset(lib):
+    """The oracle's forwards for a subset of rows (as the full-size parity tests
+    and the CPU baseline call them) equal the matching rows of the whole-batch
+    forward, for a non-contiguous, unsorted subset with a repeated row. The
+    outlier set stays a property of the whole batch: a subset without any
+    outlier row still gets the outlier product of the planted columns."""
+    w = wl.random_case(31, 23, 80, 24, n_outliers=3, frac=0.3)
+    X, W, b = _inputs(w)
+    CB, SCB = oracle.prepare_weight(W, lib=lib)
+    S = np.array([17, 2, 9, 21, 2, 0, 13], dtype=np.int64)
+    for thr in (w.threshold, math.inf):
+        full64, full16, n_full = oracle.forward(X, CB, SCB, W, thr, b, lib=lib)
+        sub64, sub16, n_sub = oracle.forward(X, CB, SCB, W, thr, b, rows=S, lib=lib)
+        assert n_sub == n_full
+        assert np.array_equal(sub64, full64[S]) and np.array_equal(sub16, full16[S])
+    # rows that hold no outlier value: O still comes from every row of X
+    O = wl.outlier_columns(w)
+    quiet = np.flatnonzero((np.abs(X[:, O].astype(np.float32)) < w.threshold).all(axis=1))
+    assert len(quiet) >= 2
+    sub64, _, n_sub = oracle.forward(X, CB, SCB, W, w.threshold, b, rows=quiet[::-1].copy(), lib=lib)
+    assert n_sub == len(O)
+    full64, _, _ = oracle.forward(X, CB, SCB, W, w.threshold, b, lib=lib)
+    assert np.array_equal(sub64, full64[quiet[::-1]])
+    QB, NDB, ZB, SB = oracle.zp_quantize_rows(W, lib=lib)
+    zfull = oracle.zp_forward(X, QB, NDB, ZB, SB, b, lib=lib)
+    zsub = oracle.zp_forward(X, QB, NDB, ZB, SB, b, rows=S, lib=lib)
+    assert np.array_equal(zsub, zfull[S])
+
+
 def _zp_rows(seed):
     """Rows for the zeropoint pins: symmetric, one-sided (ReLU-like), shifted
     far from zero, constant and all-zero rows."""
@@ -378,4 +407,4 @@ PINS = [pin_half_decode, pin_half_encode, pin_worked_example, pin_absmax_invaria
         pin_planted_outliers, pin_row_scale_excludes_outliers, pin_round_ties_to_even, pin_gemm_exact,
         pin_gemm_overflow, pin_all_columns_outlier, pin_all_columns_outlier_int8_weights,
         pin_outlier_weight_gather, pin_forward_within_bound, pin_zp_invariants, pin_zp_unrolled_product,
-        pin_zp_forward_within_bound, pin_zp_worked_examples]
+        pin_zp_forward_within_bound, pin_zp_worked_examples, pin_row_subset]

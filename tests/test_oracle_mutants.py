@@ -43,6 +43,12 @@ MUTANTS = [
     ("zp_correction_swapped", "(int64_t)ZPB[j] * sa + (int64_t)za * SUMB[j]", "(int64_t)za * sa + (int64_t)ZPB[j] * SUMB[j]"),
     ("weight_scale_wrong_row", "SCB[j] = quantize_vector(W + j * K, NULL, K, CB + j * K);",
      "SCB[j] = quantize_vector(W + j * K, NULL, K - 1, CB + j * K);"),
+    ("forward_rows_ignores_subset", "int64_t i = rows[r];", "int64_t i = r;"),
+    ("zp_forward_rows_ignores_subset", "zp_quantize_vector(X + rows[r] * K, K, ca, &za, &sa);",
+     "zp_quantize_vector(X + r * K, K, ca, &za, &sa);"),
+    ("forward_rows_outliers_from_subset",
+     "int64_t n_out = oracle_outlier_columns(X, M, K, threshold, idx);",
+     "int64_t n_out = oracle_outlier_columns(X + rows[0] * K, 1, K, threshold, idx);"),
 ]
 
 
