@@ -1,17 +1,20 @@
 """Benchmark of the LLM.int8() linear layer on B200.
 
 A step is one int8lt_forward (outlier detect + row quantize + int8 tensor-core
-GEMM with the fused dequantize / fp16 outlier product / bias epilogue) over
-the 6.7B-class projection prefill X fp16 [2048 x 4096] . W [4096 x 4096]^T
-with 6 outlier feature columns (threshold 6.0) unless --workload says
-otherwise. Inputs are resident in HBM; several input sets rotate so that the
-bytes touched between two uses of a set exceed the 126 MB L2.
+GEMM with the fused dequantize / fp16 outlier product / bias epilogue). The
+headline workload is the largest single-GPU configuration, the 175B-class
+fused QKV prefill X fp16 [8192 x 12288] . W [36864 x 12288]^T with 6 outlier
+feature columns at the threshold 6.0, unless --workload says otherwise.
+Inputs are resident in HBM; several input sets rotate so that the bytes
+touched between two uses of a set exceed the 126 MB L2.
 
 Prints ONE JSON line (rank 0). Value = effective TOPS = 2*M*N*K per forward,
 summed over ranks, over the max-over-ranks device time of the timed steps.
 The timed steps replay CUDA graphs of up to 10 whole steps without event
 nodes between kernels; each half is then timed alone over the same steps for
-the per-kernel figures (phases_ms, roofline).
+the per-kernel figures (phases_ms, roofline). The same measurement, without
+the host-buffer loop, runs on the 4096-token FFN prefill pair and the decode
+sweep (M = 1, 4, 16) and is reported under `targets`.
 Multi-GPU: one process per GPU, each runs its own replica (independent
 batches, no collective on the data path); NCCL only for the barrier and the
 max-over-ranks time.
@@ -42,16 +45,19 @@ METRIC = "int8 mixed-precision linear effective TOPS & tokens/s; % of INT8 peak 
 L2_BYTES = 126 * 1024 * 1024
 INT8_PER_BF16 = 2.0  # dense int8 / dense bf16 tensor throughput (4.5 / 2.25 PFLOP/s nominal)
 STEPS_PER_GRAPH = 10
+TARGET_MIN_STEPS = 200   # steps of each target workload reported beside the headline
 
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-targets", action="store_true",
+                   help="skip the FFN prefill and decode target workloads reported beside the headline")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--out", default=None, help="also append the JSON line to this file")
@@ -282,26 +288,38 @@ def emit(line: dict, out: str | None):
 
 # -------------------------------------------------------------- GPU bench --
 
-def run_ours(args, rank: int, world: int, local_rank: int):
+_W_CACHE: dict = {}
+
+
+def weight_of(w: wl.Workload) -> np.ndarray:
+    """W of a workload; workloads of one family (the decode sweep, the QKV sweep) share it."""
+    key = (w.wid, w.N, w.K, w.sigma_w, w.seed)
+    if key not in _W_CACHE:
+        _W_CACHE.clear()
+        _W_CACHE[key] = wl.make_w(w)
+    return _W_CACHE[key]
+
+
+def measure(args, w: wl.Workload, rank: int, world: int, local_rank: int, K_steps: int,
+            warmup: int, with_e2e: bool) -> dict:
+    """Time `K_steps` forwards of workload `w` (after `warmup` untimed ones) and each of its
+    halves alone; with_e2e adds the pipelined host-buffer loop. Returns the measurements."""
     import torch
 
-    from bit_quantized_matmul_int8_b200 import _lib, build
+    from bit_quantized_matmul_int8_b200 import _lib
 
-    build.build()
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = wl.WORKLOADS[args.workload]
     M, N, K = w.M, w.N, w.K
     N_full = N
     peaks = load_peaks()
 
     X = wl.make_x(w)
-    W = wl.make_w(w)
+    W = weight_of(w)
     b = wl.make_bias(w)
     split = args.split and world > 1
     if split:
         # This rank's output channels; X is whole on every rank.
-        from bit_quantized_matmul_int8_b200.shard import gather_shards, shard_rows
+        from bit_quantized_matmul_int8_b200.shard import shard_rows
 
         n0, n1 = shard_rows(N, world, rank)
         if n1 <= n0:
@@ -351,12 +369,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     del CB0
     stream = torch.cuda.current_stream()
 
-    def step(s):
+    for s in range(max(3, warmup)):
         r = s % R
         fwd(Xs[r], CBs[r], Ys[r], WSs[r], stream)
-
-    for s in range(max(3, args.warmup)):
-        step(s)
     torch.cuda.synchronize()
 
     # The timed steps are replayed from CUDA graphs of up to STEPS_PER_GRAPH
@@ -364,9 +379,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # event nodes inside, so consecutive kernels overlap through programmatic
     # stream serialization as they do in a model's forward. (An event node
     # between two kernels stops that overlap and costs about 9 us per step
-    # on this workload.)
+    # on the projection prefill.)
     decode = M <= 16
-    K_steps = args.steps
     cap_stream = torch.cuda.Stream(device=dev)
 
     def capture(s0, s1, quantize=True, matmul=True):
@@ -400,6 +414,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     gather = split and args.gather
     if gather:
+        from bit_quantized_matmul_int8_b200.shard import gather_shards
+
         # One graph per step; the all-gather of the Y shards runs between them.
         graphs = [capture(s0, s0 + 1) for s0 in range(K_steps)]
     else:
@@ -411,7 +427,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             if gather:
                 gather_shards(Ys[i % R], N_full)
 
-    for _ in range(max(1, math.ceil(max(3, args.warmup) / K_steps))):
+    for _ in range(max(1, math.ceil(max(3, warmup) / K_steps))):
         replay_steps()
     torch.cuda.synchronize()
 
@@ -495,6 +511,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                      if not zp else f"{alg_bytes} bytes per launch (CB + NDB/ZB/SB + CA"
                                                     f" + NDA/ZA/SA + Y)"}
 
+    out = {
+        "workload": w, "M": M, "N": N, "N_full": N_full, "K": K, "split": split, "gather": gather,
+        "R": R, "touched": touched, "keep_w": keep_w, "zp": zp, "ws_bytes": ws_bytes,
+        "steps": K_steps, "value": value, "ms_per_step": elapsed_ms / K_steps,
+        "tokens_per_s": tokens_per_s, "clocks": sampler.summary(),
+        "phases_ms": {"quantize": q_avg * 1e3, "matmul": m_avg * 1e3,
+                      "how": "each half alone over the same steps, back to back from graphs"},
+        "roofline": roof, "X": X, "W": W,
+    }
+    if not with_e2e:
+        return out
+
     # End to end through the public API, as a serving loop runs it: every step
     # copies its X in from pinned host memory, runs int8lt_forward and copies Y
     # out to pinned host memory. Copies in, compute and copies out go on three
@@ -545,37 +573,90 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_ops = 2.0 * M * N_full * K / world if split else ops  # per rank, whole job = x world
-    e2e = {"value": whole_job_rate(e2e_ops, n_e2e, world, e2e_ms) / 1e12, "unit": "TOPS",
-           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yhs[0].numel() * 2),
-           "pipeline": "copy-in / forward / copy-out on three streams, two buffer slots",
-           "steps": n_e2e, "tokens_per_s": whole_job_rate(M, n_e2e, world, e2e_ms) / (world if split else 1)}
+    out["e2e"] = {"value": whole_job_rate(e2e_ops, n_e2e, world, e2e_ms) / 1e12, "unit": "TOPS",
+                  "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yhs[0].numel() * 2),
+                  "pipeline": "copy-in / forward / copy-out on three streams, two buffer slots",
+                  "steps": n_e2e,
+                  "tokens_per_s": whole_job_rate(M, n_e2e, world, e2e_ms) / (world if split else 1)}
+    return out
+
+
+def clock_scaled(ms: float, clocks: dict) -> dict:
+    """The step time with the SM clock it ran at: ms x median MHz, and the time it
+    would take at the maximum clock if it scaled with the clock alone."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if not mhz or not mx:
+        return {}
+    return {"ms_x_sm_mhz": ms * mhz, "ms_at_max_clock": ms * mhz / mx}
+
+
+def target_summary(r: dict) -> dict:
+    """The figures of one target workload, for the JSON line's `targets` object."""
+    roof = r["roofline"]
+    d = {"ms_per_step": r["ms_per_step"], "steps": r["steps"], "value": r["value"], "unit": "TOPS",
+         "tokens_per_s": r["tokens_per_s"], "phases_ms": r["phases_ms"],
+         "dominant_kernel": {k: roof[k] for k in ("kernel", "bound", "achieved", "peak", "unit", "frac",
+                                                  "frac_of_sustained") if k in roof},
+         "clocks": r["clocks"], "clocks_while_timed": roof["clocks_while_timed"]}
+    d.update(clock_scaled(r["ms_per_step"], r["clocks"]))
+    return d
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+
+    from bit_quantized_matmul_int8_b200 import _lib, build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    w = wl.WORKLOADS[args.workload]
+    r = measure(args, w, rank, world, local_rank, args.steps, args.warmup, with_e2e=True)
+    M, N, N_full, K = r["M"], r["N"], r["N_full"], r["K"]
+    X, W = r.pop("X"), r.pop("W")
+    zp, keep_w, split = r["zp"], r["keep_w"], r["split"]
+
+    # The other target shapes, each timed the same way over its own steps (at
+    # least TARGET_MIN_STEPS, so that every timed region spans a few clock samples).
+    targets = {}
+    if not args.no_targets and not split:
+        for name in wl.TARGETS:
+            if name == w.name:
+                continue
+            torch.cuda.empty_cache()
+            t = measure(args, wl.WORKLOADS[name], rank, world, local_rank,
+                        max(args.steps, TARGET_MIN_STEPS), args.warmup, with_e2e=False)
+            targets[name] = target_summary(t)
+            del t
+    torch.cuda.empty_cache()
 
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": K_steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps, "higher_is_better": True,
+        "metric": METRIC, "value": r["value"], "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
         "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": w.name, "M": M, "K": K, "N": N_full, "n_outliers": w.n_outliers,
                    "threshold": w.threshold, "x": "N(0,1) fp16 + planted outlier columns",
-                   "w": f"N(0,{w.sigma_w}) fp16", "l2": f"{R} rotating input sets "
-                   f"({R * touched / 2**20:.0f} MiB touched per cycle) > 126 MB L2",
+                   "w": f"N(0,{w.sigma_w}) fp16", "l2": f"{r['R']} rotating input sets "
+                   f"({r['R'] * r['touched'] / 2**20:.0f} MiB touched per cycle) > 126 MB L2",
                    "parallelism": (f"N split x{world} ({N} channels per rank"
-                                   + (", Y all-gathered" if gather else "") + ")") if split
+                                   + (", Y all-gathered" if r["gather"] else "") + ")") if split
                    else f"replicas x{world}", "quant": args.quant,
                    "cuda_graphs": f"up to {STEPS_PER_GRAPH} whole steps per graph, no event nodes inside"},
-        "tokens_per_s": tokens_per_s,
+        "tokens_per_s": r["tokens_per_s"],
         "memory": {"layer_bytes": _lib.int8lt_weight_bytes(N, K) + (12 * N if zp else 4 * N)
                    + (2 * N * K if keep_w else 0),
                    "fp16_layer_bytes": 2 * N * K, "fp16_weight_kept": keep_w,
-                   "workspace_bytes": ws_bytes},
-        "phases_ms": {"quantize": q_avg * 1e3, "matmul": m_avg * 1e3,
-                      "how": "each half alone over the same steps, back to back from graphs"},
-        "roofline": roof,
-        "e2e": e2e,
-        "gpu_launches": K_steps * 2,  # the quantize kernel + the GEMM or GEMV, per step
-        "clocks": sampler.summary(),
+                   "workspace_bytes": r["ws_bytes"]},
+        "phases_ms": r["phases_ms"],
+        "roofline": r["roofline"],
+        "e2e": r["e2e"],
+        "gpu_launches": args.steps * 2,  # the quantize kernel + the GEMM or GEMV, per step
+        "clocks": r["clocks"],
     }
+    line.update({k: v for k, v in clock_scaled(r["ms_per_step"], r["clocks"]).items()})
+    if targets:
+        line["targets"] = targets
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_oracle_sample(w, args.cpu_seconds, X, W, args.quant, keep_w)
     elif not args.no_cpu_baseline:

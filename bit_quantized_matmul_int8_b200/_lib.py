@@ -27,7 +27,9 @@ EXPORTS = [
     "int8lt_status_string", "int8lt_version", "int8lt_workspace_size", "int8lt_workspace_init",
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
-    "int8lt_forward_static_scratch", "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout", "int8lt_set_gemm_split",
+    "int8lt_forward_static_scratch", "int8lt_static_scratch_read_status",
+    "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout",
+    "int8lt_debug_barrier_timeout", "int8lt_debug_static_scratch_timeout", "int8lt_set_gemm_split",
     "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
     "int8lt_forward_zp_quantize", "int8lt_forward_zp_matmul",
     "int8lt_weight_bytes", "int8lt_pack_weight", "int8lt_unpack_weight", "int8lt_layer_bytes",
@@ -58,7 +60,10 @@ _SIGS = {
     "int8lt_forward_matmul": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "int8lt_forward_static_scratch": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _F, _P, _P, _P]),
     "int8lt_debug_gemm_i32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "int8lt_static_scratch_read_status": (ctypes.c_int, [_P]),
     "int8lt_debug_wait_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
+    "int8lt_debug_barrier_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
+    "int8lt_debug_static_scratch_timeout": (ctypes.c_int, [_I64, _P]),
     "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
     "int8lt_set_gemm_split": (ctypes.c_int, [ctypes.c_int]),
     "int8lt_quantize_rows_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
@@ -114,13 +119,51 @@ def _stream(stream) -> int | None:
     return int(stream)
 
 
-def _dev(t: torch.Tensor, dtype, name: str) -> None:
-    if not t.is_cuda:
+def _dev(t: torch.Tensor, dtype, name: str, shape=None, device=None, cuda: bool = True) -> None:
+    """Check a tensor argument before it reaches the library: on a CUDA device
+    (the same one as ``device`` when given), of ``dtype``, contiguous and, when
+    ``shape`` is given, of exactly that shape."""
+    if cuda and not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the input on {device}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def forward_args(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
+                 W_outlier: torch.Tensor | None, bias: torch.Tensor | None,
+                 Y: torch.Tensor | None, cuda: bool = True) -> tuple[int, int, int]:
+    """Validate the tensors of a forward call and return (M, N, K).
+
+    X fp16 [M, K]; SCB fp32 [N]; CB the blocked codes of an [N, K] weight;
+    W_outlier fp16 [N, K] or None; bias fp16 [N] or None; Y fp16 [M, N] or
+    None. Everything on X's device. Raises ValueError before any launch, so
+    that a buffer of the wrong size never reaches a kernel.
+    """
+    if X.dim() != 2:
+        raise ValueError(f"X must be 2-D [M, K], got shape {tuple(X.shape)}")
+    M, K = X.shape
+    _dev(X, torch.float16, "X", cuda=cuda)
+    if SCB.dim() != 1:
+        raise ValueError(f"SCB must be 1-D [N], got shape {tuple(SCB.shape)}")
+    N = SCB.shape[0]
+    _dev(SCB, torch.float32, "SCB", device=X.device, cuda=cuda)
+    _dev(CB, torch.int8, "CB", device=X.device, cuda=cuda)
+    if CB.numel() != int8lt_weight_bytes(N, K):
+        raise ValueError(f"CB holds {CB.numel()} bytes; the blocked codes of a [{N},{K}] weight "
+                         f"take {int8lt_weight_bytes(N, K)}")
+    if W_outlier is not None:
+        _dev(W_outlier, torch.float16, "W_outlier", (N, K), X.device, cuda)
+    if bias is not None:
+        _dev(bias, torch.float16, "bias", (N,), X.device, cuda)
+    if Y is not None:
+        _dev(Y, torch.float16, "Y", (M, N), X.device, cuda)
+    return M, N, K
 
 
 # ------------------------------------------------------------ entry points --
@@ -227,15 +270,7 @@ def int8lt_forward(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor,
                    bias: torch.Tensor | None = None, Y: torch.Tensor | None = None,
                    ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Y fp16 [M,N] = LLM.int8() forward of X fp16 [M,K] with CB/SCB (and fp16 outlier weights)."""
-    _dev(X, torch.float16, "X")
-    _dev(SCB, torch.float32, "SCB")
-    if W_outlier is not None:
-        _dev(W_outlier, torch.float16, "W_outlier")
-    if bias is not None:
-        _dev(bias, torch.float16, "bias")
-    M, K = X.shape
-    N = SCB.shape[0]
-    _check_cb(CB, N, K)
+    M, N, K = forward_args(X, CB, SCB, W_outlier, bias, Y)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
     if ws is None:
@@ -251,8 +286,7 @@ def int8lt_forward_quantize(X: torch.Tensor, CB: torch.Tensor, SCB: torch.Tensor
                             W_outlier: torch.Tensor | None, threshold: float, ws: torch.Tensor,
                             stream=None) -> None:
     """First half of int8lt_forward: quantize X (and gather outlier weights) into ws."""
-    M, K = X.shape
-    N = SCB.shape[0]
+    M, N, K = forward_args(X, CB, SCB, W_outlier, None, None)
     _check("int8lt_forward_quantize",
            lib().int8lt_forward_quantize(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier),
                                          float(threshold), _ptr(ws), ws.numel(), _stream(stream)))
@@ -263,6 +297,13 @@ def int8lt_forward_matmul(M: int, K: int, CB: torch.Tensor, SCB: torch.Tensor,
                           Y: torch.Tensor, ws: torch.Tensor, stream=None) -> torch.Tensor:
     """Second half of int8lt_forward: GEMM/GEMV + fused epilogue from ws into Y."""
     N = SCB.shape[0]
+    _dev(Y, torch.float16, "Y", (M, N))
+    _dev(SCB, torch.float32, "SCB", (N,), Y.device)
+    _check_cb(CB, N, K)
+    if W_outlier is not None:
+        _dev(W_outlier, torch.float16, "W_outlier", (N, K), Y.device)
+    if bias is not None:
+        _dev(bias, torch.float16, "bias", (N,), Y.device)
     _check("int8lt_forward_matmul",
            lib().int8lt_forward_matmul(M, N, K, _ptr(CB), _ptr(SCB), _ptr(W_outlier), _ptr(bias),
                                        _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
@@ -279,8 +320,7 @@ def int8lt_forward_static_scratch(X: torch.Tensor, CB: torch.Tensor, SCB: torch.
     ``Y`` must be supplied (allocating it here would defeat the purpose). Calls that
     overlap on the GPU share the one array and race; order them on one stream.
     """
-    M, K = X.shape
-    N = SCB.shape[0]
+    M, N, K = forward_args(X, CB, SCB, W_outlier, bias, Y)
     _check("int8lt_forward_static_scratch",
            lib().int8lt_forward_static_scratch(_ptr(X), M, N, K, _ptr(CB), _ptr(SCB),
                                                _ptr(W_outlier), float(threshold), _ptr(bias),
@@ -306,6 +346,22 @@ def int8lt_debug_gemm_i32(CA: torch.Tensor, CB: torch.Tensor, N: int, ws: torch.
 def int8lt_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
     _check("int8lt_debug_wait_timeout",
            lib().int8lt_debug_wait_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
+
+
+def int8lt_debug_barrier_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    _check("int8lt_debug_barrier_timeout",
+           lib().int8lt_debug_barrier_timeout(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)))
+
+
+def int8lt_static_scratch_read_status(stream=None) -> int:
+    """Status of int8lt_forward_static_scratch on the current device (0 = OK,
+    7 = a kernel timed out); clears it and restores the array after a timeout."""
+    return int(lib().int8lt_static_scratch_read_status(_stream(stream)))
+
+
+def int8lt_debug_static_scratch_timeout(limit_ns: int, stream=None) -> None:
+    _check("int8lt_debug_static_scratch_timeout",
+           lib().int8lt_debug_static_scratch_timeout(int(limit_ns), _stream(stream)))
 
 
 def int8lt_quantize_rows_zp(X: torch.Tensor, stream=None):
@@ -345,15 +401,9 @@ def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: 
                       Y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
                       stream=None) -> torch.Tensor:
     """Y fp16 [M,N]: zeropoint-quantized X times the zeropoint-quantized weight, plus bias."""
-    _dev(X, torch.float16, "X")
-    _dev(NDB, torch.float32, "NDB")
-    _dev(ZB, torch.int32, "ZB")
-    _dev(SB, torch.int32, "SB")
-    if bias is not None:
-        _dev(bias, torch.float16, "bias")
-    M, K = X.shape
-    N = NDB.shape[0]
-    _check_cb(CB, N, K)
+    M, N, K = forward_args(X, CB, NDB, None, bias, Y)
+    _dev(ZB, torch.int32, "ZB", (N,), X.device)
+    _dev(SB, torch.int32, "SB", (N,), X.device)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
     if ws is None:
@@ -366,6 +416,7 @@ def int8lt_forward_zp(X: torch.Tensor, CB: torch.Tensor, NDB: torch.Tensor, ZB: 
 
 def int8lt_forward_zp_quantize(X: torch.Tensor, N: int, ws: torch.Tensor, stream=None) -> None:
     """First half of int8lt_forward_zp: zeropoint-quantize X's rows into ws."""
+    _dev(X, torch.float16, "X")
     M, K = X.shape
     _check("int8lt_forward_zp_quantize",
            lib().int8lt_forward_zp_quantize(_ptr(X), M, N, K, _ptr(ws), ws.numel(), _stream(stream)))
@@ -376,6 +427,13 @@ def int8lt_forward_zp_matmul(M: int, K: int, CB: torch.Tensor, NDB: torch.Tensor
                              ws: torch.Tensor, stream=None) -> None:
     """Second half of int8lt_forward_zp: GEMM/GEMV with the zeropoint epilogue into Y."""
     N = NDB.shape[0]
+    _dev(Y, torch.float16, "Y", (M, N))
+    _dev(NDB, torch.float32, "NDB", (N,), Y.device)
+    _dev(ZB, torch.int32, "ZB", (N,), Y.device)
+    _dev(SB, torch.int32, "SB", (N,), Y.device)
+    _check_cb(CB, N, K)
+    if bias is not None:
+        _dev(bias, torch.float16, "bias", (N,), Y.device)
     _check("int8lt_forward_zp_matmul",
            lib().int8lt_forward_zp_matmul(M, N, K, _ptr(CB), _ptr(NDB), _ptr(ZB), _ptr(SB),
                                           _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(),

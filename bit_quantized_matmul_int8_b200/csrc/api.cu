@@ -447,4 +447,14 @@ int int8lt_debug_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void 
     return from_cuda(launch_wait_timeout(&hdr->status, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
+int int8lt_debug_barrier_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream) {
+    if (!ws) return INT8LT_ERR_NULL;
+    if (ws_bytes < kWsInitBytes) return INT8LT_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return INT8LT_ERR_ALIGN;
+    if (limit_ns < 1000 || limit_ns > 1000000000) return INT8LT_ERR_VALUE;
+    if (int st = check_device()) return st;
+    return from_cuda(launch_barrier_timeout(static_cast<WsHeader *>(ws), (uint64_t)limit_ns,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -178,6 +178,8 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t
               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 cudaError_t launch_wait_timeout(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
+// One CTA at the quantize pass's grid barrier, waiting for a CTA that does not exist.
+cudaError_t launch_barrier_timeout(WsHeader *h, uint64_t limit_ns, cudaStream_t s);
 
 // The two halves of int8lt_forward on an already validated call; `ws` holds
 // at least ws_layout(M, N, K).total bytes. Return an int8lt_status.

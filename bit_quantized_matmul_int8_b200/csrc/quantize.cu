@@ -317,18 +317,20 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
 }
 
 // Grid-wide barrier of the cooperative launch. The arrival count only grows:
-// this launch's CTAs are all in once it reaches base + gridDim.x, which the
-// waiters see directly in the count. The last CTA in publishes the next
-// launch's base and generation (no CTA of this launch reads them any more;
-// the next launch, behind this one in stream order, does). Every wait is
-// bounded; after a timeout the count is off and the workspace header must be
-// initialised again. Returns false (and records a timeout) if it ran out.
-__device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base) {
+// this launch's `ctas` CTAs (its grid) are all in once it reaches base +
+// ctas, which the waiters see directly in the count. The last CTA in
+// publishes the next launch's base and generation (no CTA of this launch
+// reads them any more; the next launch, behind this one in stream order,
+// does). Every wait is bounded by limit_ns; after a timeout the count is off
+// and the workspace header must be initialised again. Returns false (and
+// records a timeout) if it ran out.
+__device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base, uint32_t ctas,
+                             uint64_t limit_ns = kWaitLimitNs) {
     __shared__ uint32_t s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t ok = 1;
-        const uint32_t target = base + gridDim.x;
+        const uint32_t target = base + ctas;
         __threadfence();
         const uint32_t old = atomicAdd(&h->bar_count, 1u);
         if (old == target - 1u) {
@@ -337,7 +339,7 @@ __device__ bool grid_barrier(WsHeader *h, uint32_t gen, uint32_t base) {
         } else {
             const uint64_t t0 = globaltimer_ns();
             while ((int32_t)(ld_acquire_u32(&h->bar_count) - target) < 0) {
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                if (globaltimer_ns() - t0 > limit_ns) {
                     ok = 0;
                     record_timeout(&h->status);
                     break;
@@ -440,7 +442,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
     if (!alone) {
         for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
             if (bits[w]) atomicOr(&cur[w], bits[w]);
-        if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
+        if (!grid_barrier(a.hdr, gen, s_base, gridDim.x)) return;  // every CTA waits in the same barrier
     }
 
     // Phase B: codes, scales, outlier activations; outlier-weight gather.
@@ -720,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     }
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
         if (bits[w]) atomicOr(&cur[w], bits[w]);
-    if (!grid_barrier(a.hdr, gen, s_base)) return;  // every CTA waits in the same barrier
+    if (!grid_barrier(a.hdr, gen, s_base, gridDim.x)) return;  // every CTA waits in the same barrier
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
         uint32_t v = __ldcg(&cur[w]);
         if (w == kwords - 1 && (a.K & 31)) v &= (1u << (a.K & 31)) - 1u;
@@ -862,6 +864,21 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
             }
         }
     }
+}
+
+// Test kernel: the quantize pass's grid barrier, entered by a grid that
+// counts one CTA more than it has, so the wait cannot end before limit_ns.
+// It reads the launch generation and base as quantize_kernel does, records
+// the timeout in the status word and returns; the header's counts are then
+// off until the workspace is initialised again.
+__global__ void barrier_timeout_kernel(WsHeader *h, uint64_t limit_ns) {
+    __shared__ uint32_t s_gen, s_base;
+    if (threadIdx.x == 0) {
+        s_gen = *reinterpret_cast<volatile uint32_t *>(&h->qgen);
+        s_base = *reinterpret_cast<volatile uint32_t *>(&h->qbase);
+    }
+    __syncthreads();
+    grid_barrier(h, s_gen, s_base, gridDim.x + 1u, limit_ns);
 }
 
 }  // namespace
@@ -1020,6 +1037,11 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, quantize_kernel, a, kwords, R, rounds);
+}
+
+cudaError_t launch_barrier_timeout(WsHeader *h, uint64_t limit_ns, cudaStream_t s) {
+    barrier_timeout_kernel<<<1, kThreads, 0, s>>>(h, limit_ns);
+    return cudaGetLastError();
 }
 
 }  // namespace int8lt

@@ -19,10 +19,17 @@
 // different host threads) race on the array and corrupt each other.
 //
 // In host code `g_scratch` is only a host-side stand-in for the device
-// symbol, not a device address. The device address is taken once per device
-// with cudaGetSymbolAddress, with that device current, on the first call the
-// process makes on that device; that first call should therefore come before
-// any stream capture.
+// symbol, not a device address. The device address is taken with
+// cudaGetSymbolAddress, with the device current, on the first call the
+// process makes on that device, which also zeroes the whole array with a
+// synchronous cudaMemset; that first call should therefore come before any
+// stream capture. Only a successful set-up is kept: if it fails (for example
+// because a capture is under way), the call reports INT8LT_ERR_CUDA and the
+// next call on that device tries again.
+//
+// Device-side timeouts land in the array's own status word, which callers
+// read (and clear) with int8lt_static_scratch_read_status.
+#include <atomic>
 #include <mutex>
 
 #include "int8lt_internal.cuh"
@@ -34,26 +41,40 @@ constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_setup_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_setup_err[kMaxDevices];
+std::mutex g_setup_mu;
+std::atomic<void *> g_scratch_ptr[kMaxDevices];
 
 // Device address of g_scratch on the current device (set up on first use).
 int scratch_on_current_device(void **ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return INT8LT_ERR_CUDA;
-    std::call_once(g_setup_once[dev], [dev] {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-        // Start from a zeroed scratch (as int8lt_workspace_init leaves a
-        // workspace); synchronous, once.
-        if (e == cudaSuccess) e = cudaMemset(p, 0, kStaticScratchBytes);
-        g_setup_err[dev] = e;
-        g_scratch_ptr[dev] = (e == cudaSuccess) ? p : nullptr;
-    });
-    if (g_setup_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return INT8LT_ERR_CUDA;
-    *ptr = g_scratch_ptr[dev];
+    void *p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_setup_mu);
+        p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            // Start from a zeroed array, as int8lt_workspace_init leaves a
+            // workspace. On failure clear the runtime's last error, so that a
+            // later launch check does not report this call's failure again.
+            if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p ||
+                cudaMemset(p, 0, kStaticScratchBytes) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return INT8LT_ERR_CUDA;
+            }
+            g_scratch_ptr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *ptr = p;
     return INT8LT_OK;
+}
+
+int device_supported() {
+    int major = 0, minor = 0, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return INT8LT_ERR_CUDA;
+    return (major == 10 && minor == 0) ? INT8LT_OK : INT8LT_ERR_UNSUPPORTED;
 }
 
 bool is_aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -73,15 +94,45 @@ extern "C" int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N
         (W_outlier && !is_aligned(W_outlier, 16)) || (bias && !is_aligned(bias, 2)))
         return INT8LT_ERR_ALIGN;
     if (threshold != threshold || threshold < 0.f) return INT8LT_ERR_VALUE;
-    int major = 0, minor = 0, dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return INT8LT_ERR_CUDA;
-    if (major != 10 || minor != 0) return INT8LT_ERR_UNSUPPORTED;
+    if (int st = device_supported()) return st;
     void *ws = nullptr;
     if (int st = scratch_on_current_device(&ws)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (int st = forward_quantize(X, M, N, K, CB, SCB, W_outlier, threshold, ws, s)) return st;
     return forward_matmul(M, N, K, CB, SCB, W_outlier, bias, Y, ws, s);
+}
+
+// Synchronize the stream, then read the array's status word on the current
+// device. A timeout also re-zeroes the header and the column bitmaps (the
+// barrier counts of the quantize pass may be off after one), which is what
+// int8lt_workspace_init does for a workspace; every other part of the array
+// is rewritten by each call.
+extern "C" int int8lt_static_scratch_read_status(void *stream) {
+    using namespace int8lt;
+    if (int st = device_supported()) return st;
+    void *ws = nullptr;
+    if (int st = scratch_on_current_device(&ws)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t status = 0;
+    if (cudaMemcpyAsync(&status, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return INT8LT_ERR_CUDA;
+    if (status == 0) return INT8LT_OK;
+    if (cudaMemsetAsync(ws, 0, kWsInitBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        return INT8LT_ERR_CUDA;
+    return (status & kStatusTimeout) ? INT8LT_ERR_TIMEOUT : INT8LT_ERR_CUDA;
+}
+
+// Test entry: the quantize pass's grid-barrier wait run out against the
+// array's header, as a real timeout would leave it.
+extern "C" int int8lt_debug_static_scratch_timeout(int64_t limit_ns, void *stream) {
+    using namespace int8lt;
+    if (limit_ns < 1000 || limit_ns > 1000000000) return INT8LT_ERR_VALUE;
+    if (int st = device_supported()) return st;
+    void *ws = nullptr;
+    if (int st = scratch_on_current_device(&ws)) return st;
+    return launch_barrier_timeout(static_cast<WsHeader *>(ws), (uint64_t)limit_ns,
+                                  static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? INT8LT_OK
+               : INT8LT_ERR_CUDA;
 }

@@ -80,8 +80,15 @@ for _w in [
 ] + [_qkv(o, t) for o in (0, 6, 24, 246) for t in (6.0, math.inf)]:
     WORKLOADS[_w.name] = _w
 
-# The workload the headline number is quoted on (6.7B-class projection prefill).
-HEADLINE = "proj_prefill_2048x4096x4096"
+# The workload the headline number is quoted on: the largest single-GPU
+# configuration, the 175B-class fused QKV prefill with 6 outlier columns at
+# the threshold 6.0.
+HEADLINE = "qkv_prefill_8192x12288x36864_o6_t6"
+
+# Reported beside the headline: the 4096-token FFN prefill pair (tensor-bound)
+# and the decode GEMV sweep (HBM-bound).
+TARGETS = ("ffn_up_4096x4096x16384", "ffn_down_4096x16384x4096", "decode_m1_12288x49152",
+           "decode_m4_12288x49152", "decode_m16_12288x49152")
 
 _T_X, _T_OUTCOLS, _T_OUTROWS, _T_OUTVAL, _T_W, _T_BIAS = range(6)
 

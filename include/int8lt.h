@@ -222,17 +222,35 @@ int int8lt_forward_matmul(int64_t M, int64_t N, int64_t K, const int8_t *CB, con
  *     must fit the 8 MiB array (e.g. K = 12288 with N up to about 100k);
  *     larger calls return INT8LT_ERR_TOO_LARGE without launching anything.
  *   - The array lives on every GPU on which the library is loaded, until the
- *     process exits. The first call on a device looks up the array's device
- *     address (with that device current) and clears its header; make that
- *     first call before any stream capture.
+ *     process exits. The first call on a device (this one or
+ *     int8lt_static_scratch_read_status) looks up the array's device address
+ *     with that device current and zeroes the whole array with a synchronous
+ *     cudaMemset; make that first call before any stream capture. If that
+ *     set-up fails, the call returns INT8LT_ERR_CUDA and the next call tries
+ *     again.
  *   - All calls on a device share the array. Each call re-initialises what
  *     it reads, but calls whose kernels overlap on the GPU (unordered streams
  *     or concurrent host threads) race on it and produce wrong results.
+ *   - A bounded wait that runs out on the device is recorded in the array's
+ *     own status word, not reported by this call's return value: read it
+ *     with int8lt_static_scratch_read_status (the output of a call that timed
+ *     out is undefined).
  * Other arguments and errors as int8lt_forward.
  */
 int int8lt_forward_static_scratch(const void *X, int64_t M, int64_t N, int64_t K,
                                   const int8_t *CB, const float *SCB, const void *W_outlier,
                                   float threshold, const void *bias, void *Y, void *stream);
+
+/*
+ * Device status of int8lt_forward_static_scratch on the current device, as
+ * int8lt_read_device_status is for a workspace: synchronizes `stream`, reads
+ * and clears the fixed array's status word, and returns INT8LT_OK, or
+ * INT8LT_ERR_TIMEOUT if a kernel of an earlier call gave up a bounded wait
+ * (after which the array's header and bitmaps are zeroed again, so the next
+ * call starts clean), or INT8LT_ERR_CUDA if the stream reported an error.
+ * Allocates nothing.
+ */
+int int8lt_static_scratch_read_status(void *stream);
 
 /* ------------------------------------------------- zeropoint quantization -- */
 
@@ -346,6 +364,26 @@ int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int mode, int32_t 
  * hang is involved.
  */
 int int8lt_debug_wait_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream);
+
+/*
+ * Test entry: one block enters the grid-wide barrier of the quantize pass
+ * (the step between outlier detection and quantization) of a launch that
+ * counts one block more than it has, so its bounded wait gives up after
+ * `limit_ns` nanoseconds (1e3 .. 1e9). The kernel records INT8LT_ERR_TIMEOUT
+ * in the workspace status word and returns normally. The barrier's counts in
+ * the workspace header are then off, as after any such timeout: call
+ * int8lt_workspace_init before the workspace's next use. ws_bytes must cover
+ * the header and bitmaps (any int8lt_workspace_size of a valid shape does).
+ */
+int int8lt_debug_barrier_timeout(void *ws, size_t ws_bytes, int64_t limit_ns, void *stream);
+
+/*
+ * Test entry: as int8lt_debug_barrier_timeout, against the header of the
+ * fixed array of int8lt_forward_static_scratch on the current device, so that
+ * int8lt_static_scratch_read_status can be seen to report the timeout and
+ * restore the array.
+ */
+int int8lt_debug_static_scratch_timeout(int64_t limit_ns, void *stream);
 
 #ifdef __cplusplus
 }

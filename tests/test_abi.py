@@ -98,6 +98,92 @@ def test_other_entry_validation(L):
     assert L.int8lt_debug_wait_timeout(None, 4096, 10000, None) == E["INT8LT_ERR_NULL"]
     assert L.int8lt_workspace_init(None, 4096, None) == E["INT8LT_ERR_NULL"]
     assert L.int8lt_read_device_status(FAKE, 16, None) == E["INT8LT_ERR_WORKSPACE"]
+    bt = L.int8lt_debug_barrier_timeout
+    assert bt(None, 1 << 20, 10000, None) == E["INT8LT_ERR_NULL"]
+    assert bt(FAKE, 256, 10000, None) == E["INT8LT_ERR_WORKSPACE"]   # header only: no bitmaps
+    assert bt(FAKE + 8, 1 << 20, 10000, None) == E["INT8LT_ERR_ALIGN"]
+    assert bt(FAKE, 1 << 20, 10, None) == E["INT8LT_ERR_VALUE"]
+    assert bt(FAKE, 1 << 20, 2_000_000_000, None) == E["INT8LT_ERR_VALUE"]
+    assert L.int8lt_debug_static_scratch_timeout(10, None) == E["INT8LT_ERR_VALUE"]
+
+
+def _cpu_forward_tensors(M=4, N=64, K=128):
+    import torch
+    X = torch.zeros((M, K), dtype=torch.float16)
+    CB = torch.zeros(_lib.int8lt_weight_bytes(N, K), dtype=torch.int8)
+    SCB = torch.zeros(N, dtype=torch.float32)
+    W = torch.zeros((N, K), dtype=torch.float16)
+    b = torch.zeros(N, dtype=torch.float16)
+    Y = torch.zeros((M, N), dtype=torch.float16)
+    return X, CB, SCB, W, b, Y
+
+
+def test_binding_accepts_consistent_forward_arguments(L):
+    X, CB, SCB, W, b, Y = _cpu_forward_tensors()
+    assert _lib.forward_args(X, CB, SCB, W, b, Y, cuda=False) == (4, 64, 128)
+    assert _lib.forward_args(X, CB, SCB, None, None, None, cuda=False) == (4, 64, 128)
+
+
+@pytest.mark.parametrize("bad", ["Y_short", "Y_wide", "Y_dtype", "Y_strided", "Y_1d", "CB_other_layer",
+                                 "W_outlier_shape", "bias_shape", "SCB_dtype", "X_dtype", "X_3d"])
+def test_binding_rejects_mismatched_forward_arguments(L, bad):
+    """A buffer of the wrong size, type or layout raises in the binding, before
+    any call into the library (so before any launch, with or without a GPU)."""
+    import torch
+    X, CB, SCB, W, b, Y = _cpu_forward_tensors()
+    if bad == "Y_short":
+        Y = torch.zeros((3, 64), dtype=torch.float16)
+    elif bad == "Y_wide":
+        Y = torch.zeros((4, 72), dtype=torch.float16)
+    elif bad == "Y_dtype":
+        Y = torch.zeros((4, 64), dtype=torch.float32)
+    elif bad == "Y_strided":
+        Y = torch.zeros((64, 4), dtype=torch.float16).t()
+    elif bad == "Y_1d":
+        Y = torch.zeros(4 * 64, dtype=torch.float16)
+    elif bad == "CB_other_layer":
+        CB = torch.zeros(_lib.int8lt_weight_bytes(64, 256), dtype=torch.int8)
+    elif bad == "W_outlier_shape":
+        W = torch.zeros((64, 64), dtype=torch.float16)
+    elif bad == "bias_shape":
+        b = torch.zeros(32, dtype=torch.float16)
+    elif bad == "SCB_dtype":
+        SCB = torch.zeros(64, dtype=torch.float16)
+    elif bad == "X_dtype":
+        X = torch.zeros((4, 128), dtype=torch.float32)
+    elif bad == "X_3d":
+        X = torch.zeros((1, 4, 128), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        _lib.forward_args(X, CB, SCB, W, b, Y, cuda=False)
+
+
+def test_binding_forward_wrappers_validate_first(L, monkeypatch):
+    """The forward wrappers run the checks above before they touch the library:
+    with the library calls replaced by a recorder, a wrong Y raises and nothing
+    is recorded."""
+    import torch
+    calls = []
+
+    class Recorder:
+        def __getattr__(self, name):
+            return lambda *a: calls.append(name) or 0
+
+    real = _lib.lib()
+    weight_bytes = lambda N, K: int(real.int8lt_weight_bytes(N, K))  # noqa: E731 (host query)
+    dev_check = _lib._dev
+    monkeypatch.setattr(_lib, "lib", lambda path=None: Recorder())
+    monkeypatch.setattr(_lib, "int8lt_weight_bytes", weight_bytes)
+    # CPU tensors stand in for device ones: every check but "is it on a GPU" runs
+    monkeypatch.setattr(_lib, "_dev", lambda t, dtype, name, shape=None, device=None, cuda=True:
+                        dev_check(t, dtype, name, shape, device, False))
+    X, CB, SCB, W, b, _ = _cpu_forward_tensors()
+    Y = torch.zeros((3, 64), dtype=torch.float16)
+    for call in (lambda: _lib.int8lt_forward(X, CB, SCB, W, 6.0, b, Y=Y),
+                 lambda: _lib.int8lt_forward_static_scratch(X, CB, SCB, W, Y, 6.0, b),
+                 lambda: _lib.int8lt_forward_matmul(4, 128, CB, SCB, W, b, Y, X)):
+        with pytest.raises(ValueError, match="Y has shape"):
+            call()
+    assert calls == []
 
 
 def test_zeropoint_entry_validation(L):

@@ -361,6 +361,32 @@ def test_bounded_wait_reports_timeout():
     assert len(idx) == 2
 
 
+def test_grid_barrier_timeout_is_reported_and_recoverable():
+    """The quantize pass's grid-barrier wait, run out on purpose (a launch that
+    counts one block more than it has, 1 ms limit): the workspace status reports
+    INT8LT_ERR_TIMEOUT once, and after int8lt_workspace_init the next forwards
+    through the same workspace equal the ones before."""
+    w = wl.random_case(72, 300, 1024, 256, n_outliers=3, frac=0.5)
+    X, W, b = case_inputs(w)
+    Xd, Wd, bd = dev(X), dev(W), dev(b)
+    CB, SCB = _lib.int8lt_prepare_weight(Wd)
+    ws = _lib.workspace(w.M, w.N, w.K)
+    ref = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, ws=ws).clone()
+    assert _lib.int8lt_read_device_status(ws) == 0
+    _lib.int8lt_debug_barrier_timeout(ws, 1_000_000)
+    assert _lib.int8lt_read_device_status(ws) == _lib.STATUS_CODE["INT8LT_ERR_TIMEOUT"]
+    assert _lib.int8lt_read_device_status(ws) == 0           # the read cleared it
+    _lib.int8lt_workspace_init(ws)
+    for _ in range(2):
+        Y = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, ref)
+    assert _lib.int8lt_read_device_status(ws) == 0
+    CBo, SCBo = oracle.prepare_weight(W)
+    Y64, _, _ = oracle.forward(X, CBo, SCBo, W, 6.0, b)
+    check_y(host(ref), Y64, "forward around the barrier timeout")
+
+
 def test_validation_errors_raise():
     W = dev(wl.make_w(wl.random_case(71, 1, 64, 64)))
     CB, SCB = _lib.int8lt_prepare_weight(W)

@@ -36,6 +36,9 @@ def test_inf_threshold_keeps_data():
 def test_headline_and_configs():
     assert wl.HEADLINE in wl.WORKLOADS
     h = wl.WORKLOADS[wl.HEADLINE]
-    assert (h.M, h.K, h.N, h.n_outliers) == (2048, 4096, 4096, 6)
+    # the largest single-GPU configuration: the fused QKV prefill at threshold 6.0
+    assert (h.M, h.K, h.N, h.n_outliers, h.threshold) == (8192, 12288, 36864, 6, 6.0)
+    assert h.ops == max(w.ops for w in wl.WORKLOADS.values())
+    assert all(t in wl.WORKLOADS and t != wl.HEADLINE for t in wl.TARGETS)
     assert wl.WORKLOADS["ffn_down_4096x16384x4096"].n_outliers == 12
     assert wl.WORKLOADS["qkv_prefill_8192x12288x36864_o246_t6"].n_outliers == 246
