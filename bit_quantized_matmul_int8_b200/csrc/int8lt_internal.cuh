@@ -59,6 +59,7 @@ struct WsHeader {
     uint32_t qbase;        // bar_count when the next quantize launch starts
     uint32_t pad[59];
 };
+static_assert(sizeof(WsHeader) == 256, "workspace header");
 constexpr size_t kWsBitmapOffset = 1024;
 // Stream-K of the prefill GEMM: one ready flag per (CTA pair, rank) in the
 // zeroed region, and one int32 partial tile (128 x 256) per (pair, rank).

@@ -81,6 +81,11 @@ QCASES = [
     ("long_ragged", wl.random_case(48, 610, 10256, 8, n_outliers=5, frac=0.4), None),
     # rows too long to keep in shared memory: read from X in both phases
     ("very_long_rows", wl.random_case(47, 20, 65536, 8, n_outliers=3, frac=0.5), None),
+    # decode batches (M <= 16): column slices of one cluster, staged or not
+    ("decode_one_row", wl.random_case(49, 1, 12288, 8, n_outliers=6, frac=1.0), None),
+    ("decode_ragged", wl.random_case(50, 7, 4112, 8, n_outliers=9, frac=0.5), None),
+    ("decode_full", wl.random_case(51, 16, 12288, 8, n_outliers=24, frac=0.75), None),
+    ("decode_max_k", wl.random_case(52, 16, 133136, 8, n_outliers=5, frac=0.5), None),
 ]
 
 
@@ -99,7 +104,7 @@ def test_quantize_rows_bit_exact(name, w, _, thr):
 
 
 @pytest.mark.parametrize("M,K", [(40, 256), (300, 1040), (2048, 4096), (17, 4096), (40, 8192), (33, 8208),
-                                 (300, 16384), (700, 12288)])
+                                 (300, 16384), (700, 12288), (7, 64), (16, 12288), (9, 133136)])
 def test_quantize_row_max_in_other_rows_outlier_column(M, K):
     """A row whose largest magnitude sits in a column that only other rows make an
     outlier: its scale must come from the columns outside O (a ([P] decomposition)
@@ -385,6 +390,36 @@ def test_grid_barrier_timeout_is_reported_and_recoverable():
     CBo, SCBo = oracle.prepare_weight(W)
     Y64, _, _ = oracle.forward(X, CBo, SCBo, W, 6.0, b)
     check_y(host(ref), Y64, "forward around the barrier timeout")
+
+
+def test_workspace_shared_across_shapes():
+    """One workspace, large enough for each call, serves calls of different
+    shapes in turn (decode batches of several sizes, a prefill batch, the
+    zeropoint forward): each result equals the same call on a fresh workspace."""
+    cases = [wl.random_case(74, 16, 4096, 1024, n_outliers=3, frac=1.0),
+             wl.random_case(75, 4, 1024, 2056, n_outliers=2, frac=1.0),
+             wl.random_case(76, 300, 1024, 1024, n_outliers=4, frac=0.5),
+             wl.random_case(77, 9, 4096, 1024, n_outliers=3, frac=1.0),
+             wl.random_case(74, 16, 4096, 1024, n_outliers=3, frac=1.0)]
+    size = max(_lib.int8lt_workspace_size(c.M, c.N, c.K) for c in cases)
+    shared = torch.empty(size, dtype=torch.uint8, device="cuda")
+    _lib.int8lt_workspace_init(shared)
+    for i, c in enumerate(cases):
+        X, W, b = case_inputs(c)
+        Xd, Wd, bd = dev(X), dev(W), dev(b)
+        CB, SCB = _lib.int8lt_prepare_weight(Wd)
+        ref = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd)
+        for _ in range(2):
+            Y = _lib.int8lt_forward(Xd, CB, SCB, Wd, 6.0, bd, ws=shared)
+            torch.cuda.synchronize()
+            assert torch.equal(Y, ref), (i, c.name)
+        if c.M <= 16:   # the zeropoint decode forward on the same workspace
+            CBz, NDB, ZB, SB = _lib.int8lt_prepare_weight_zp(Wd)
+            refz = _lib.int8lt_forward_zp(Xd, CBz, NDB, ZB, SB, bd)
+            Yz = _lib.int8lt_forward_zp(Xd, CBz, NDB, ZB, SB, bd, ws=shared)
+            torch.cuda.synchronize()
+            assert torch.equal(Yz, refz), (i, c.name, "zeropoint")
+    assert _lib.int8lt_read_device_status(shared) == 0
 
 
 def test_validation_errors_raise():
