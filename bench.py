@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--sets", type=int, default=0,
+                   help="rotating input sets (default: enough that a cycle touches 3x the L2); "
+                        "1 keeps the device memory small, e.g. for a profiler capture")
     p.add_argument("--no-targets", action="store_true",
                    help="skip the FFN prefill and decode target workloads reported beside the headline")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -362,6 +365,8 @@ def measure(args, w: wl.Workload, rank: int, world: int, local_rank: int, K_step
     ws_bytes = _lib.int8lt_workspace_size(M, N, K)
     touched = X.nbytes + M * K + (M * N * 2) + M * K + N * K  # X + CA + Y + CB(+CA write)
     R = int(min(16, max(3, math.ceil(3 * L2_BYTES / touched))))
+    if getattr(args, "sets", 0) > 0:
+        R = int(args.sets)
     Xs = [Xh.to(dev) for _ in range(R)]
     CBs = [CB0.clone() for _ in range(R)]
     Ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for _ in range(R)]

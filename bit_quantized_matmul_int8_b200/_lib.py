@@ -14,11 +14,15 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libint8lt.so")
+# The same library built with -DINT8LT_DEBUG: its kernels check the index of
+# every computed global access and report a failed check as INT8LT_ERR_BOUNDS.
+CHECK_LIB_PATH = os.path.join(_HERE, "libint8lt_check.so")
 
 STATUS = {
     0: "INT8LT_OK", 1: "INT8LT_ERR_NULL", 2: "INT8LT_ERR_SHAPE", 3: "INT8LT_ERR_ALIGN",
     4: "INT8LT_ERR_VALUE", 5: "INT8LT_ERR_WORKSPACE", 6: "INT8LT_ERR_CUDA",
     7: "INT8LT_ERR_TIMEOUT", 8: "INT8LT_ERR_UNSUPPORTED", 9: "INT8LT_ERR_TOO_LARGE",
+    10: "INT8LT_ERR_BOUNDS",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -90,6 +94,27 @@ def lib(path: str | None = None) -> ctypes.CDLL:
                                    "`python -m bit_quantized_matmul_int8_b200.build`")
             _lib = _bind(ctypes.CDLL(LIB_PATH))
     return _lib
+
+
+class using_library:
+    """Context manager: route this module's calls to another build of the
+    library (e.g. CHECK_LIB_PATH) inside the block; not for concurrent use."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        lib()                       # the regular library, loaded once
+        with _lock:
+            self.saved = _lib
+            _lib = _bind(ctypes.CDLL(self.path))
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self.saved
 
 
 def _bind(l: ctypes.CDLL) -> ctypes.CDLL:

@@ -189,6 +189,7 @@ const char *int8lt_status_string(int status) {
         case INT8LT_ERR_UNSUPPORTED: return "INT8LT_ERR_UNSUPPORTED: device is not compute capability 10.0";
         case INT8LT_ERR_TOO_LARGE:
             return "INT8LT_ERR_TOO_LARGE: M > 16 or the call's scratch exceeds the 8 MiB static array";
+        case INT8LT_ERR_BOUNDS: return "INT8LT_ERR_BOUNDS: a kernel index failed its bounds check";
         default: return "INT8LT_ERR_UNKNOWN";
     }
 }
@@ -220,7 +221,8 @@ int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream) {
     if (status == 0) return INT8LT_OK;
     if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return INT8LT_ERR_CUDA;
-    return (status & kStatusTimeout) ? INT8LT_ERR_TIMEOUT : INT8LT_ERR_CUDA;
+    if (status & kStatusTimeout) return INT8LT_ERR_TIMEOUT;
+    return (status & kStatusBounds) ? INT8LT_ERR_BOUNDS : INT8LT_ERR_CUDA;
 }
 
 size_t int8lt_weight_bytes(int64_t N, int64_t K) {

@@ -90,6 +90,25 @@ struct TileSched {
     }
 };
 
+// Output tile t -> (tile row m, tile column n). The tiles go in groups of
+// kGroupM tile rows, tile column by tile column inside a group, so the pairs
+// working at the same time (one wave of consecutive tiles) share a few row
+// panels of A and column panels of B; the next wave reuses the same A panels
+// from L2. (With the tile row as the fast index a wave touched every row panel
+// of A, and on a 8192 x 12288 x 36864 product the kernel read 8.1 GB from DRAM
+// for 0.55 GB of operands.)
+constexpr int kGroupM = 8;
+__host__ __device__ __forceinline__ void tile_mn(int t, int num_m, int num_tiles, int &m, int &n) {
+    const int num_n = num_tiles / num_m;
+    const int per_group = kGroupM * num_n;
+    const int g = t / per_group;
+    const int first_m = g * kGroupM;
+    const int gm = min(num_m - first_m, kGroupM);
+    const int r = t - g * per_group;
+    m = first_m + r % gm;
+    n = r / gm;
+}
+
 // Split policy (INT8LT_SPLIT_*): process-wide, read at each launch.
 std::atomic<int> g_split_mode{0};
 
@@ -364,7 +383,8 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // reads what the quantize pass wrote (launched with programmatic stream
     // serialization, the prologue overlaps the end of that pass).
     grid_dep_wait();
-    const int n_out = (!kZp && a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
+    int n_out = (!kZp && a.n_outliers && a.Xo && a.Wo && !a.C32) ? *a.n_outliers : 0;
+    if (!IN_BOUNDS(n_out >= 0 && n_out <= a.kcap, a.status)) n_out = 0;
     const int n_okb = (n_out + kOkb - 1) / kOkb;       // outlier k-blocks per tile
     const int n_mma_o = (n_out + 15) >> 4;             // fp16 MMAs of K = 16 per tile
     const uint32_t tmem = ctrl->tmem_base;
@@ -405,8 +425,10 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const uint32_t fb = smem_u32(&ctrl->ofull);
                     if (rank == 0) mbar_arrive_expect_tx(fb, kOTxBytes);
                     const uint32_t fb_leader = mapa_shared(fb, 0);
-                    const int32_t m0 = (gp.tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
-                    const int32_t n0 = (gp.tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
+                    int tm, tn;
+                    tile_mn(gp.tile, num_m_tiles, num_tiles, tm, tn);
+                    const int32_t m0 = tm * BM + (int32_t)rank * kCtaRows;
+                    const int32_t n0 = tn * BN + (int32_t)rank * kCtaRows;
                     tma_load_2d_pair(smem_u32(sXo), &tmXo, fb_leader, okb * kOkb, m0);
                     tma_load_2d_pair(smem_u32(sWo), &tmWo, fb_leader, okb * kOkb, n0);
                     ++o_issued;
@@ -420,8 +442,10 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             TileSched ts(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
             Seg g;
             while (!*abort_flag && ts.next(g)) {
-                const int32_t m0 = (g.tile % num_m_tiles) * BM + (int32_t)rank * kCtaRows;
-                const int32_t n0 = (g.tile / num_m_tiles) * BN + (int32_t)rank * kCtaRows;
+                int tm, tn;
+                tile_mn(g.tile, num_m_tiles, num_tiles, tm, tn);
+                const int32_t m0 = tm * BM + (int32_t)rank * kCtaRows;
+                const int32_t n0 = tn * BN + (int32_t)rank * kCtaRows;
                 for (int kb = g.kb0; kb < g.kb1; ++kb) {
                     if (*abort_flag) break;
                     const uint32_t eb = smem_u32(&ctrl->empty[stage]);
@@ -572,8 +596,10 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         TileSched ts(num_tiles, nkb, nkb, num_pairs, pair, sk_on);
         Seg g;
         for (; ts.next(g); ++it) {
-            const int64_t m0 = (int64_t)(g.tile % num_m_tiles) * BM + rank * kCtaRows;
-            const int64_t n0 = (int64_t)(g.tile / num_m_tiles) * BN;
+            int tm, tn;
+            tile_mn(g.tile, num_m_tiles, num_tiles, tm, tn);
+            const int64_t m0 = (int64_t)tm * BM + rank * kCtaRows;
+            const int64_t n0 = (int64_t)tn * BN;
             const int buf = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             // Fetch this tile's column data (thread et owns column n0 + et)
@@ -668,7 +694,7 @@ gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     int32_t *dst = a.C32 + row * a.N + c0;
 #pragma unroll
                     for (int v = 0; v < 8; ++v)
-                        if (c0 + 4 * v < a.N)
+                        if (c0 + 4 * v < a.N && IN_BOUNDS(row * a.N + c0 + 4 * v + 3 < a.M * a.N, a.status))
                             reinterpret_cast<int4 *>(dst)[v] = make_int4((int)acc[4 * v], (int)acc[4 * v + 1],
                                                                          (int)acc[4 * v + 2], (int)acc[4 * v + 3]);
                 }

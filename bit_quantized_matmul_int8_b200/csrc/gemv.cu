@@ -68,6 +68,7 @@ __device__ __forceinline__ uint4 ld_stream(const int8_t *p) {
 }
 
 __device__ __forceinline__ float outlier_weight(const GemvArgs &a, int64_t j, int64_t col) {
+    if (!IN_BOUNDS(col >= 0 && col < a.K, a.status)) return 0.f;
     if (a.W_outlier) return __half2float(a.W_outlier[j * a.K + col]);
     const float p = __fmul_rn((float)a.CB[cb_offset(j, col, wblocks_k(a.K))], a.SCB[j]);
     return __half2float(__float2half_rn(__fdiv_rn(p, 127.f)));
@@ -135,6 +136,7 @@ __device__ __forceinline__ void row_block_out(const GemvArgs &a, int n_out, int6
         for (int hi = 0; hi < 2; ++hi) {
             const int64_t t = g + hi * 8, j = n0 + 8 * q + 2 * tig;
             if (t >= a.M || j >= a.N) continue;  // N % 8 == 0: j + 1 < N too
+            if (!IN_BOUNDS(t * a.N + j + 1 < a.M * a.N, a.status)) continue;
             const int32_t c0 = d[q][2 * hi], c1 = d[q][2 * hi + 1];
             if (a.C32) {
                 *reinterpret_cast<int2 *>(a.C32 + t * a.N + j) = make_int2(c0, c1);
@@ -180,7 +182,8 @@ gemv_i8_kernel(const GemvArgs a, const int64_t L) {
     const bool tok_lo = g < a.M, tok_hi = kHi && g + 8 < a.M;
     const int8_t *xa = a.CA + (int64_t)g * a.K;
     const int8_t *xb = a.CA + (int64_t)(g + 8) * a.K;
-    const int n_out = kOut ? *a.n_outliers : 0;
+    int n_out = kOut ? *a.n_outliers : 0;
+    if (!IN_BOUNDS(n_out >= 0 && n_out <= a.kcap, a.status)) n_out = 0;
     const uint4 z = make_uint4(0, 0, 0, 0);
     // This lane's 16-byte pieces of a block: rows 8q + g, bytes 64h + 16tig.
     const int lane_off = g * kWBlockCols + tig * (kWide ? 32 : 16);
@@ -233,11 +236,12 @@ gemv_i8_kernel(const GemvArgs a, const int64_t L) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int64_t t = g + (e >> 1) * 8, j = n0 + 8 * q + 2 * tig + (e & 1);
-                    if (t < a.M && j < a.N) atomicAdd(&a.acc[j * a.M + t], d[q][e]);
+                    if (t < a.M && j < a.N && IN_BOUNDS(j * a.M + t < a.N * a.M, a.status))
+                        atomicAdd(&a.acc[j * a.M + t], d[q][e]);
                 }
             __threadfence();
             uint32_t old = 0;
-            if (lane == 0) old = atomicAdd(&a.cnt[rb], 1u);
+            if (lane == 0 && IN_BOUNDS(rb < ceil_div(a.N, 8), a.status)) old = atomicAdd(&a.cnt[rb], 1u);
             old = __shfl_sync(0xffffffffu, old, 0);
             mine = old == (uint32_t)(w_last - w_first);
             if (mine) {

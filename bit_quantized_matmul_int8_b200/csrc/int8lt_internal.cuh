@@ -18,6 +18,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s bound on every in-kerne
 
 // Device status bits (workspace header word 0).
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBounds = 2u;  // checking builds: an index failed its bounds check
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
@@ -250,6 +251,21 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 __device__ __forceinline__ void record_timeout(uint32_t *status) {
     if (status) atomicOr(status, kStatusTimeout);
 }
+
+// Bounds checks of the checking build (compiled with -DINT8LT_DEBUG): every
+// computed global access of the kernels goes through IN_BOUNDS(index <
+// extent, status word); a failed check records kStatusBounds and the access
+// is skipped, so a wrong index is reported instead of touching memory that is
+// not the buffer's. The regular build compiles the checks away.
+__device__ __forceinline__ bool bounds_ok(bool ok, uint32_t *status) {
+    if (!ok && status) atomicOr(status, kStatusBounds);
+    return ok;
+}
+#ifdef INT8LT_DEBUG
+#define IN_BOUNDS(cond, status) (::int8lt::bounds_ok((cond), (status)))
+#else
+#define IN_BOUNDS(cond, status) true
+#endif
 
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

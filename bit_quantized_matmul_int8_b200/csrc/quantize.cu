@@ -215,15 +215,17 @@ __device__ __forceinline__ uint4 clear_masked(uint4 x, uint32_t m) {
 }
 
 // Xo[rank of column] = x for the outlier elements (bits of m) of vector v.
+// `cap` is the row's capacity in Xo; `st` the status word of a checking build.
 __device__ __forceinline__ void store_outliers(uint4 x, uint32_t m, int v, const uint32_t *bits,
-                                               const int32_t *prefix, __half *xo) {
+                                               const int32_t *prefix, __half *xo, int64_t cap, uint32_t *st) {
     while (m) {
         const int j = __ffs(m) - 1;
         m &= m - 1;
         const uint32_t w = j < 4 ? (j < 2 ? x.x : x.y) : (j < 6 ? x.z : x.w);
         const unsigned short h = (unsigned short)((j & 1) ? (w >> 16) : (w & 0xffffu));
         const int col = v * 8 + j;
-        xo[prefix[col >> 5] + __popc(bits[col >> 5] & ((1u << (col & 31)) - 1u))] = __ushort_as_half(h);
+        const int64_t rank = prefix[col >> 5] + __popc(bits[col >> 5] & ((1u << (col & 31)) - 1u));
+        if (IN_BOUNDS(rank >= 0 && rank < cap, st)) xo[rank] = __ushort_as_half(h);
     }
 }
 
@@ -260,14 +262,15 @@ __device__ __forceinline__ void quantize_row(const QuantizeArgs &a, const uint4 
         uint4 x = ld_vec<kSmem>(row + v);
         const uint32_t m = vec_mask(bits, v);
         if (m) {
-            if (xo) store_outliers(x, m, v, bits, prefix, xo);
+            if (xo) store_outliers(x, m, v, bits, prefix, xo, a.kcap, &a.hdr->status);
             x = clear_masked(x, m);
         }
         ca2[v] = quant_vec8(x, s);
     }
     if (xo) {
         const int32_t n16 = (n_out + 15) & ~15;
-        for (int32_t t = n_out + lane; t < n16; t += 32) xo[t] = __float2half_rn(0.f);
+        for (int32_t t = n_out + lane; t < n16; t += 32)
+            if (IN_BOUNDS(t < a.kcap, &a.hdr->status)) xo[t] = __float2half_rn(0.f);
     }
     if (lane == 0) a.SCA[r] = sa;
 }
@@ -461,7 +464,8 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
                 uint32_t v = bits[w];
                 int32_t r = prefix[w];
                 while (v) {
-                    a.outlier_idx[r++] = (int32_t)(w * 32 + __ffs(v) - 1);
+                    if (IN_BOUNDS(r >= 0 && r < a.K, &a.hdr->status)) a.outlier_idx[r] = (int32_t)(w * 32 + __ffs(v) - 1);
+                    ++r;
                     v &= v - 1;
                 }
             }
@@ -483,7 +487,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
         for (int u = 0; u < 4; ++u) {
             const int64_t j = j0 + u * nhw;
             gv[u] = __float2half_rn(0.f);
-            if (real && j < a.N) {
+            if (real && j < a.N && IN_BOUNDS(col >= 0 && col < a.K, &a.hdr->status)) {
                 if (a.W_outlier) {
                     gv[u] = a.W_outlier[j * a.K + col];
                 } else {
@@ -497,7 +501,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int64_t j = j0 + u * nhw;
-            if (j < a.N) a.Wo[j * a.kcap + t0 + hl] = gv[u];
+            if (j < a.N && IN_BOUNDS(t0 + hl < a.kcap, &a.hdr->status)) a.Wo[j * a.kcap + t0 + hl] = gv[u];
         }
     };
     const bool gather = a.Wo && n16 > 0;
@@ -545,7 +549,7 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
                     val = rh[col];
                     rh[col] = __ushort_as_half((unsigned short)0);
                 }
-                if (xo) xo[t] = val;
+                if (xo && IN_BOUNDS(t < a.kcap, &a.hdr->status)) xo[t] = val;
             }
             __syncwarp();
             if (!long_rows) quantize_row_plain(a, rows + (size_t)r * nvec, r0 + r, lane);
@@ -738,7 +742,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
                 uint32_t v = bits[w];
                 int32_t rk = prefix[w];
                 while (v) {
-                    a.outlier_idx[rk++] = (int32_t)(w * 32 + __ffs(v) - 1);
+                    if (IN_BOUNDS(rk >= 0 && rk < a.K, &a.hdr->status)) a.outlier_idx[rk] = (int32_t)(w * 32 + __ffs(v) - 1);
+                    ++rk;
                     v &= v - 1;
                 }
             }
@@ -781,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
             if (j >= nrows) break;
             const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
             if (lane < n_out) a.CA[r * a.K + col] = 0;
-            if (a.Xo && lane < n16) a.Xo[r * a.kcap + lane] = vals[i];
+            if (a.Xo && lane < n16 && IN_BOUNDS(lane < a.kcap, &a.hdr->status)) a.Xo[r * a.kcap + lane] = vals[i];
         }
     } else {
         for (int j = warp; j < nrows; j += kWarps) {
@@ -793,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
                     val = a.X[r * a.K + col];
                     a.CA[r * a.K + col] = 0;
                 }
-                if (a.Xo) a.Xo[r * a.kcap + t] = val;
+                if (a.Xo && IN_BOUNDS(t < a.kcap, &a.hdr->status)) a.Xo[r * a.kcap + t] = val;
             }
         }
     }
@@ -852,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
             const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
             for (int64_t jj = hw; jj < a.N; jj += nhw) {
                 __half g = __float2half_rn(0.f);
-                if (real) {
+                if (real && IN_BOUNDS(col >= 0 && col < a.K, &a.hdr->status)) {
                     if (a.W_outlier) {
                         g = a.W_outlier[jj * a.K + col];
                     } else {
@@ -860,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
                         g = __float2half_rn(__fdiv_rn(p, 127.f));
                     }
                 }
-                a.Wo[jj * a.kcap + t] = g;
+                if (IN_BOUNDS(t < a.kcap, &a.hdr->status)) a.Wo[jj * a.kcap + t] = g;
             }
         }
     }
@@ -1027,7 +1032,7 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
             const int32_t n16 = (n_out + 15) & ~15;
             for (int i = threadIdx.x; i < M * (n16 - n_out); i += kThreads) {
                 const int t = i / (n16 - n_out), j = n_out + i % (n16 - n_out);
-                a.Xo[(int64_t)t * a.kcap + j] = __float2half_rn(0.f);
+                if (IN_BOUNDS(j < a.kcap, &a.hdr->status)) a.Xo[(int64_t)t * a.kcap + j] = __float2half_rn(0.f);
             }
         }
     }
@@ -1036,7 +1041,8 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
             uint32_t b = s_bits[i];
             int32_t r = before + s_prefix[i];
             while (b) {
-                a.outlier_idx[r++] = (int32_t)((w0 + i) * 32 + __ffs(b) - 1);
+                if (IN_BOUNDS(r >= 0 && r < a.K, &a.hdr->status)) a.outlier_idx[r] = (int32_t)((w0 + i) * 32 + __ffs(b) - 1);
+                ++r;
                 b &= b - 1;
             }
         }
@@ -1050,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
             uint4 x = kStage ? src[v] : __ldg(src + v);
             const uint32_t mk = vec_mask(s_bits, (int)v);
             if (mk) {
-                if (xo) store_outliers(x, mk, (int)v, s_bits, s_prefix, xo);
+                if (xo) store_outliers(x, mk, (int)v, s_bits, s_prefix, xo, a.kcap - before, &a.hdr->status);
                 x = clear_masked(x, mk);
             }
             ca2[v] = quant_vec8(x, sc);

@@ -120,7 +120,8 @@ extern "C" int int8lt_static_scratch_read_status(void *stream) {
     if (status == 0) return INT8LT_OK;
     if (cudaMemsetAsync(ws, 0, kWsInitBytes, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return INT8LT_ERR_CUDA;
-    return (status & kStatusTimeout) ? INT8LT_ERR_TIMEOUT : INT8LT_ERR_CUDA;
+    if (status & kStatusTimeout) return INT8LT_ERR_TIMEOUT;
+    return (status & kStatusBounds) ? INT8LT_ERR_BOUNDS : INT8LT_ERR_CUDA;
 }
 
 // Test entry: the quantize pass's grid-barrier wait run out against the

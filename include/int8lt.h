@@ -72,8 +72,11 @@ typedef enum {
     INT8LT_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
     INT8LT_ERR_TIMEOUT = 7,     /* a kernel gave up a bounded wait (device status) */
     INT8LT_ERR_UNSUPPORTED = 8, /* current device is not compute capability 10.0 */
-    INT8LT_ERR_TOO_LARGE = 9    /* call exceeds the fixed scratch of
+    INT8LT_ERR_TOO_LARGE = 9,   /* call exceeds the fixed scratch of
                                    int8lt_forward_static_scratch */
+    INT8LT_ERR_BOUNDS = 10      /* checking build only (libint8lt_check.so): a
+                                   kernel's index failed its bounds check and
+                                   the access was skipped (device status) */
 } int8lt_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -108,7 +111,8 @@ int int8lt_workspace_init(void *ws, size_t ws_bytes, void *stream);
  * Synchronize `stream`, then read and clear the workspace's status word.
  * Returns INT8LT_OK, or INT8LT_ERR_TIMEOUT if any kernel that used this
  * workspace since the last read gave up a bounded wait (its outputs are then
- * undefined), or INT8LT_ERR_CUDA if the stream reported an error.
+ * undefined), INT8LT_ERR_BOUNDS (checking build only) if a kernel's index
+ * failed its bounds check, or INT8LT_ERR_CUDA if the stream reported an error.
  */
 int int8lt_read_device_status(void *ws, size_t ws_bytes, void *stream);
 

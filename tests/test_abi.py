@@ -35,6 +35,17 @@ def test_exports_every_declared_symbol(L):
         assert getattr(L, n) is not None
 
 
+def test_checking_build_exports_every_declared_symbol(L):
+    """The checking build (-DINT8LT_DEBUG) is built beside the regular one and
+    offers the same C ABI; its extra status code has a name."""
+    assert os.path.exists(_lib.CHECK_LIB_PATH)
+    C = _lib.lib(_lib.CHECK_LIB_PATH)
+    for n in declared_symbols():
+        assert getattr(C, n) is not None
+    assert C.int8lt_status_string(10).decode().startswith("INT8LT_ERR_BOUNDS")
+    assert C.int8lt_version() == L.int8lt_version()
+
+
 def test_status_strings(L):
     for code, name in _lib.STATUS.items():
         assert L.int8lt_status_string(code).decode().startswith(name)
