@@ -58,7 +58,8 @@ struct WsHeader {
     uint32_t qgen;         // quantize launches so far: selects this launch's bitmap
     uint32_t bar_count;    // arrivals at the quantize grid barrier, all launches (wraps)
     uint32_t qbase;        // bar_count when the next quantize launch starts
-    uint32_t pad[59];
+    uint32_t row_next;     // streaming quantize: rows handed out past the first one per CTA (0 between launches)
+    uint32_t pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header");
 constexpr size_t kWsBitmapOffset = 1024;

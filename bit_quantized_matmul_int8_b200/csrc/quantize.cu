@@ -578,8 +578,10 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
 // ------------------------------------------------ streaming, row per CTA --
 //
 // For batches with long rows (see launch_quantize) X is read from HBM once:
-// each CTA streams its rows, one row at a time across its 256 threads (three
-// CTAs per SM, so one CTA's loads are in flight while the others quantize). A row's
+// each CTA streams rows, one row at a time across its 256 threads (three
+// CTAs per SM, so one CTA's loads are in flight while the others quantize);
+// after its first row a CTA takes the next untaken row from a counter in the
+// workspace header, so the rows spread by speed, not by count. A row's
 // elements with |x| >= threshold are outliers whatever the other rows hold,
 // so they are zeroed and the row's absmax and codes are taken over the rest
 // before the batch's outlier set O is known. After the grid barrier, with O
@@ -587,6 +589,8 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
 // code 0 and their values go to Xo; the absmax stands unless every element
 // attaining it lies in O (the row's maximum falls in another row's outlier
 // column), in which case the row is quantized again from X with O masked.
+// Which elements of one vector attain the absmax is recorded while the row is
+// in registers, so that check needs no second read of X.
 // Same results as quantize_kernel, bit for bit.
 constexpr int kStreamVpt = 8;                                  // 16-byte vectors per thread and row
 constexpr int64_t kStreamMaxK = (int64_t)kStreamVpt * kThreads * 8;  // 16384
@@ -621,7 +625,7 @@ __device__ __forceinline__ void stream_load(uint4 (&x)[kStreamVpt], const uint4 
 // rest, codes to CA. Records the absmax and a vector attaining it.
 __device__ __forceinline__ void stream_row(const QuantizeArgs &a, uint4 (&x)[kStreamVpt], int64_t r, int j, int nvec,
                                            uint32_t t2, uint32_t *bits, uint32_t (*s_wmax)[kWarps],
-                                           int (*s_wv)[kWarps], uint32_t *s_amax, int32_t *s_vmax) {
+                                           int (*s_wv)[kWarps], uint32_t *s_amax, int32_t *s_vmax, uint32_t *s_eqm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t mx = 0;
     int mv = 0;
@@ -669,6 +673,17 @@ __device__ __forceinline__ void stream_row(const QuantizeArgs &a, uint4 (&x)[kSt
         const int v = threadIdx.x + kThreads * i;
         if (v < nvec) ca2[v] = quant_vec8(x[i], sc);
     }
+    // The elements of vector vmax that attain the absmax (its own outliers are
+    // zero here, so they never match a nonzero absmax), from the thread that
+    // holds that vector.
+    if ((vmax & (kThreads - 1)) == (int)threadIdx.x) {
+        const int idx = vmax / kThreads;
+        uint4 xv = x[0];
+#pragma unroll
+        for (int i = 1; i < kStreamVpt; ++i)
+            if (i == idx) xv = x[i];
+        s_eqm[j] = elem_eq_mask(xv, amax);
+    }
     if (threadIdx.x == 0) {
         s_amax[j] = amax;
         s_vmax[j] = vmax;
@@ -681,7 +696,11 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     __shared__ int s_wv[2][kWarps];
     __shared__ uint32_t s_amax[kStreamMaxRows];
     __shared__ int32_t s_vmax[kStreamMaxRows];
+    __shared__ uint32_t s_eqm[kStreamMaxRows];
     __shared__ uint32_t s_gen, s_base;
+    __shared__ int32_t s_row[kStreamMaxRows];  // the rows this CTA took, in order
+    __shared__ int32_t s_next;
+    uint32_t *row_next = &a.hdr->row_next;
     const int64_t kwords = ceil_div(a.K, 32);
     uint32_t *bits = smem;                                         // [kwords]
     int32_t *prefix = reinterpret_cast<int32_t *>(smem + kwords);  // [kwords]
@@ -689,11 +708,10 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     const int nvec = (int)(a.K / 8);
     const uint32_t t2 = (uint32_t)a.tbits | ((uint32_t)a.tbits << 16);
     const uint4 *X4 = reinterpret_cast<const uint4 *>(a.X);
-    const int nrows = a.M > blockIdx.x ? (int)ceil_div(a.M - blockIdx.x, gridDim.x) : 0;
     grid_dep_launch();
 
     uint4 xa[kStreamVpt];
-    stream_load(xa, X4 + (int64_t)blockIdx.x * nvec, nvec, nrows > 0);
+    stream_load(xa, X4 + (int64_t)blockIdx.x * nvec, nvec, blockIdx.x < a.M);
     if (threadIdx.x == 0) {
         s_gen = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qgen);
         s_base = *reinterpret_cast<volatile uint32_t *>(&a.hdr->qbase);
@@ -706,11 +724,28 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < kMaxKwords; i += (int64_t)gridDim.x * kThreads)
         nxt[i] = 0;
 
-    // Rows blockIdx.x + j * gridDim.x, one at a time.
-    for (int j = 0; j < nrows; ++j) {
-        const int64_t r0 = blockIdx.x + (int64_t)j * gridDim.x;
-        if (j > 0) stream_load(xa, X4 + r0 * nvec, nvec, true);
-        stream_row(a, xa, r0, j, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax);
+    // Row blockIdx.x first, then rows taken one at a time from a shared
+    // counter (the next one is taken while the current one is quantized), so
+    // that CTAs which run faster do more rows. At most kStreamMaxRows per CTA;
+    // the launch gives every CTA room for ceil(M / grid) rows, so the others
+    // take what one CTA leaves.
+    int nrows = 0;
+    {
+        int64_t r0 = blockIdx.x;
+        for (int j = 0; r0 < a.M; ++j) {
+            if (j > 0) stream_load(xa, X4 + r0 * nvec, nvec, true);
+            const bool more = j + 1 < kStreamMaxRows;
+            uint32_t taken = 0;
+            if (threadIdx.x == 0 && more) taken = atomicAdd(row_next, 1u);
+            stream_row(a, xa, r0, j, nvec, t2, bits, s_wmax, s_wv, s_amax, s_vmax, s_eqm);
+            if (threadIdx.x == 0) {
+                s_row[j] = (int32_t)r0;
+                s_next = more ? (int32_t)min((int64_t)gridDim.x + (int64_t)taken, a.M) : (int32_t)a.M;
+            }
+            __syncthreads();
+            r0 = s_next;
+            nrows = j + 1;
+        }
     }
     __syncthreads();
 
@@ -727,6 +762,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
         if (bits[w]) atomicOr(&cur[w], bits[w]);
     if (!grid_barrier(a.hdr, gen, s_base, gridDim.x)) return;  // every CTA waits in the same barrier
+    if (blockIdx.x == 0 && threadIdx.x == 0) *row_next = 0u;  // every row has been taken
     for (int64_t w = threadIdx.x; w < kwords; w += kThreads) {
         uint32_t v = __ldcg(&cur[w]);
         if (w == kwords - 1 && (a.K & 31)) v &= (1u << (a.K & 31)) - 1u;
@@ -750,6 +786,44 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
         }
     }
 
+    // Outlier-weight gather Wo[j, t] (as quantize_kernel): half-warps over
+    // output channels, a lane per outlier rank, kGatherBatch channels' loads in
+    // flight per lane; the first batch's loads are issued here and stored
+    // after the rows are finished.
+    constexpr int kGatherBatch = 8;
+    const int hl = lane & 15;
+    const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
+    const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
+    const int64_t KB = wblocks_k(a.K);
+    __half gv[kGatherBatch];
+    auto gather_load = [&](int32_t t0, int64_t j0) {
+        const int32_t t = t0 + hl;
+        const bool real = t < n_out;
+        const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
+#pragma unroll
+        for (int u = 0; u < kGatherBatch; ++u) {
+            const int64_t jj = j0 + u * nhw;
+            gv[u] = __float2half_rn(0.f);
+            if (real && jj < a.N && IN_BOUNDS(col >= 0 && col < a.K, &a.hdr->status)) {
+                if (a.W_outlier) {
+                    gv[u] = a.W_outlier[jj * a.K + col];
+                } else {
+                    const float p = __fmul_rn((float)a.CB[cb_offset(jj, col, KB)], a.SCB[jj]);
+                    gv[u] = __float2half_rn(__fdiv_rn(p, 127.f));
+                }
+            }
+        }
+    };
+    auto gather_store = [&](int32_t t0, int64_t j0) {
+#pragma unroll
+        for (int u = 0; u < kGatherBatch; ++u) {
+            const int64_t jj = j0 + u * nhw;
+            if (jj < a.N && IN_BOUNDS(t0 + hl < a.kcap, &a.hdr->status)) a.Wo[jj * a.kcap + t0 + hl] = gv[u];
+        }
+    };
+    const bool gather = a.Wo && n16 > 0;
+    if (gather) gather_load(0, hw);
+
     // Finish the rows, a warp per row (rows warp, warp + 8, ...). Lane l first
     // checks whether row warp + 8 l keeps its absmax: some element outside O
     // attains it (else the row's maximum lies in O and the row is redone).
@@ -761,12 +835,8 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     uint32_t keep = 1;
     {
         const int j = warp + kWarps * lane;
-        if (lane < kRowsPerWarp && j < nrows && s_amax[j] != 0u) {
-            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
-            const uint4 xv = __ldg(X4 + r * nvec + s_vmax[j]);
-            const uint32_t own = flags8(ge_bits(xv.x, t2), ge_bits(xv.y, t2), ge_bits(xv.z, t2), ge_bits(xv.w, t2));
-            keep = (elem_eq_mask(xv, s_amax[j]) & ~own & ~vec_mask(bits, s_vmax[j])) != 0u;
-        }
+        if (lane < kRowsPerWarp && j < nrows && s_amax[j] != 0u)
+            keep = (s_eqm[j] & ~vec_mask(bits, s_vmax[j])) != 0u;
     }
     const uint32_t keep_mask = __ballot_sync(0xffffffffu, keep);
     // Columns of O: code 0 and the fp16 value into Xo (zero-padded to 16). With
@@ -777,20 +847,20 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) {
             const int j = warp + kWarps * i;
-            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            const int64_t r = (int64_t)s_row[j];
             vals[i] = (j < nrows && lane < n_out) ? a.X[r * a.K + col] : __float2half_rn(0.f);
         }
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) {
             const int j = warp + kWarps * i;
             if (j >= nrows) break;
-            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            const int64_t r = (int64_t)s_row[j];
             if (lane < n_out) a.CA[r * a.K + col] = 0;
             if (a.Xo && lane < n16 && IN_BOUNDS(lane < a.kcap, &a.hdr->status)) a.Xo[r * a.kcap + lane] = vals[i];
         }
     } else {
         for (int j = warp; j < nrows; j += kWarps) {
-            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            const int64_t r = (int64_t)s_row[j];
             for (int32_t t = lane; t < n16; t += 32) {
                 __half val = __float2half_rn(0.f);
                 if (t < n_out) {
@@ -804,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     }
     for (int i = 0, j = warp; j < nrows; ++i, j += kWarps) {
         if ((keep_mask >> i) & 1u) {
-            if (lane == 0) a.SCA[blockIdx.x + (int64_t)j * gridDim.x] = __half2float(__ushort_as_half((unsigned short)s_amax[j]));
+            if (lane == 0) a.SCA[(int64_t)s_row[j]] = __half2float(__ushort_as_half((unsigned short)s_amax[j]));
         } else if (lane == 0) {
             s_redo[atomicAdd(&s_nredo, 1)] = j;
         }
@@ -815,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
     const int nredo = s_nredo;
     for (int k = 0; k < nredo; ++k) {
         const int j = s_redo[k];
-        const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+        const int64_t r = (int64_t)s_row[j];
         stream_load(xa, X4 + r * nvec, nvec, true);
         uint32_t mx = 0;
 #pragma unroll
@@ -845,29 +915,13 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
         if (threadIdx.x == 0) a.SCA[r] = sa;
     }
 
-    // Outlier-weight gather Wo[j, t] (as quantize_kernel).
-    if (a.Wo && n16 > 0) {
-        const int hl = lane & 15;
-        const int64_t hw = ((int64_t)blockIdx.x * kWarps + warp) * 2 + (lane >> 4);
-        const int64_t nhw = (int64_t)gridDim.x * kWarps * 2;
-        const int64_t KB = wblocks_k(a.K);
-        for (int32_t t0 = 0; t0 < n16; t0 += 16) {
-            const int32_t t = t0 + hl;
-            const bool real = t < n_out;
-            const int64_t col = real ? outlier_column(bits, prefix, kwords, t) : 0;
-            for (int64_t jj = hw; jj < a.N; jj += nhw) {
-                __half g = __float2half_rn(0.f);
-                if (real && IN_BOUNDS(col >= 0 && col < a.K, &a.hdr->status)) {
-                    if (a.W_outlier) {
-                        g = a.W_outlier[jj * a.K + col];
-                    } else {
-                        const float p = __fmul_rn((float)a.CB[cb_offset(jj, col, KB)], a.SCB[jj]);
-                        g = __float2half_rn(__fdiv_rn(p, 127.f));
-                    }
-                }
-                if (IN_BOUNDS(t < a.kcap, &a.hdr->status)) a.Wo[jj * a.kcap + t] = g;
+    if (gather) {
+        gather_store(0, hw);
+        for (int32_t t0 = 0; t0 < n16; t0 += 16)
+            for (int64_t j0 = hw + (t0 == 0 ? kGatherBatch * nhw : 0); j0 < a.N; j0 += kGatherBatch * nhw) {
+                gather_load(t0, j0);
+                gather_store(t0, j0);
             }
-        }
     }
 }
 

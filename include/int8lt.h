@@ -99,7 +99,7 @@ size_t int8lt_workspace_size(int64_t M, int64_t N, int64_t K);
 /*
  * Prepare a freshly allocated workspace (stream-ordered): zeroes all
  * ws_bytes of it, so that the device status word, the outlier count, the
- * quantize pass's launch and barrier counters, its column bitmaps and the
+ * quantize pass's launch, barrier and row counters, its column bitmaps and the
  * prefill GEMM's split-tile flags start at zero. Call once after allocating
  * a workspace, before its first use; later calls keep it consistent by
  * themselves. After a reported INT8LT_ERR_TIMEOUT call it again before the
