@@ -394,12 +394,17 @@ def test_grid_barrier_timeout_is_reported_and_recoverable():
 
 def test_workspace_shared_across_shapes():
     """One workspace, large enough for each call, serves calls of different
-    shapes in turn (decode batches of several sizes, a prefill batch, the
-    zeropoint forward): each result equals the same call on a fresh workspace."""
+    shapes in turn (decode batches of several sizes, prefill batches of short
+    rows and of long rows, whose pass hands rows out from a counter in the
+    workspace, the zeropoint forward): each result equals the same call on a
+    fresh workspace, twice in a row."""
     cases = [wl.random_case(74, 16, 4096, 1024, n_outliers=3, frac=1.0),
              wl.random_case(75, 4, 1024, 2056, n_outliers=2, frac=1.0),
              wl.random_case(76, 300, 1024, 1024, n_outliers=4, frac=0.5),
+             wl.random_case(78, 2000, 8192, 256, n_outliers=5, frac=0.75),
+             wl.random_case(79, 300, 12288, 520, n_outliers=2, frac=0.5),
              wl.random_case(77, 9, 4096, 1024, n_outliers=3, frac=1.0),
+             wl.random_case(78, 2000, 8192, 256, n_outliers=5, frac=0.75),
              wl.random_case(74, 16, 4096, 1024, n_outliers=3, frac=1.0)]
     size = max(_lib.int8lt_workspace_size(c.M, c.N, c.K) for c in cases)
     shared = torch.empty(size, dtype=torch.uint8, device="cuda")
