@@ -442,6 +442,16 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.CB + off), "r"(n) : "memory");
         }
     }
+    // Decode path: zero the GEMV's partial sums and k-block counters here,
+    // before the barrier, where the stores overlap the wait (nothing in this
+    // pass reads them, and the GEMV reads them only after the whole pass).
+    {
+        const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x, nth = (int64_t)gridDim.x * kThreads;
+        if (a.acc)
+            for (int64_t i = tid; i < a.acc_words / 4; i += nth) reinterpret_cast<int4 *>(a.acc)[i] = make_int4(0, 0, 0, 0);
+        if (a.cnt)
+            for (int64_t i = tid; i < a.cnt_words / 4; i += nth) reinterpret_cast<uint4 *>(a.cnt)[i] = make_uint4(0, 0, 0, 0);
+    }
     if (!alone) {
         for (int64_t w = threadIdx.x; w < kwords; w += kThreads)
             if (bits[w]) atomicOr(&cur[w], bits[w]);
@@ -567,12 +577,6 @@ quantize_kernel(QuantizeArgs a, int64_t kwords, int R, int rounds) {
                 gather_store(t0, j0);
             }
     }
-    // Decode path: zero the GEMV's partial sums and k-block counters.
-    const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x, nth = (int64_t)gridDim.x * kThreads;
-    if (a.acc)
-        for (int64_t i = tid; i < a.acc_words / 4; i += nth) reinterpret_cast<int4 *>(a.acc)[i] = make_int4(0, 0, 0, 0);
-    if (a.cnt)
-        for (int64_t i = tid; i < a.cnt_words / 4; i += nth) reinterpret_cast<uint4 *>(a.cnt)[i] = make_uint4(0, 0, 0, 0);
 }
 
 // ------------------------------------------------ streaming, row per CTA --
@@ -877,40 +881,45 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_stream_kernel(QuantizeAr
             if (lane == 0) a.SCA[(int64_t)s_row[j]] = __half2float(__ushort_as_half((unsigned short)s_amax[j]));
         } else if (lane == 0) {
             s_redo[atomicAdd(&s_nredo, 1)] = j;
+            // its row is read again below: start pulling it into L2 now
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(X4 + (int64_t)s_row[j] * nvec),
+                         "r"((uint32_t)(nvec * 16)) : "memory");
         }
     }
     __syncthreads();
     // Rows whose maximum lies in O: the whole CTA quantizes them again from X
     // with O masked (rare: a row's maximum in another row's outlier column).
+    // Rolled loops that read the row again (from L2) rather than registers:
+    // this code runs about once per launch, in one CTA, and with its loops
+    // unrolled most of its time went to fetching its instructions.
     const int nredo = s_nredo;
     for (int k = 0; k < nredo; ++k) {
         const int j = s_redo[k];
         const int64_t r = (int64_t)s_row[j];
-        stream_load(xa, X4 + r * nvec, nvec, true);
+        const uint4 *row = X4 + r * nvec;
         uint32_t mx = 0;
-#pragma unroll
-        for (int i = 0; i < kStreamVpt; ++i) {
-            const int v = threadIdx.x + kThreads * i;
-            if (v < nvec) {
-                const uint32_t m = vec_mask(bits, v) | flags8(ge_bits(xa[i].x, t2), ge_bits(xa[i].y, t2),
-                                                              ge_bits(xa[i].z, t2), ge_bits(xa[i].w, t2));
-                if (m) xa[i] = clear_masked(xa[i], m);
-                mx = max(mx, vec_absmax_bits(xa[i]));
-            }
+#pragma unroll 1
+        for (int v = threadIdx.x; v < nvec; v += kThreads) {
+            uint4 x = __ldg(row + v);
+            const uint32_t m = vec_mask(bits, v);  // O holds every element at or above the threshold
+            if (m) x = clear_masked(x, m);
+            mx = max(mx, vec_absmax_bits(x));
         }
         mx = warp_max_u32(mx);
         if (lane == 0) s_wmax[k & 1][warp] = mx;
         __syncthreads();
         uint32_t amax = s_wmax[k & 1][0];
-#pragma unroll
+#pragma unroll 1
         for (int w = 1; w < kWarps; ++w) amax = max(amax, s_wmax[k & 1][w]);
         const float sa = __half2float(__ushort_as_half((unsigned short)amax));
         const float sc = sa > 0.f ? __fdiv_rn(127.f, sa) : 0.f;
         uint2 *ca2 = reinterpret_cast<uint2 *>(a.CA + r * a.K);
-#pragma unroll
-        for (int i = 0; i < kStreamVpt; ++i) {
-            const int v = threadIdx.x + kThreads * i;
-            if (v < nvec) ca2[v] = quant_vec8(xa[i], sc);
+#pragma unroll 1
+        for (int v = threadIdx.x; v < nvec; v += kThreads) {
+            uint4 x = __ldg(row + v);
+            const uint32_t m = vec_mask(bits, v);
+            if (m) x = clear_masked(x, m);
+            ca2[v] = quant_vec8(x, sc);
         }
         if (threadIdx.x == 0) a.SCA[r] = sa;
     }
@@ -1167,6 +1176,7 @@ constexpr int kQuantDynMax = 113 * 1024 - 512;
 // are quantized by a single CTA.
 constexpr int64_t kAloneElems = 64 * 1024;
 constexpr int64_t kAloneClearWords = 64 * 1024;  // and at most this many decode sums to zero
+constexpr int64_t kClearWordsPerCta = 8 * 1024;  // decode sums zeroed per CTA otherwise
 
 struct QuantOcc {
     std::mutex mu;
@@ -1358,7 +1368,9 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s) {
     // The outlier-weight gather runs over all N output channels: give it
     // enough CTAs even when there are few rows.
     if (a.Wo) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.N, 32)));
-    if (a.acc) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.acc_words, kAloneClearWords)));
+    // The decode GEMV's partial sums are zeroed 32 KB per CTA (a grid of a
+    // dozen CTAs for 3 MB took 2.5 µs longer per decode step).
+    if (a.acc) grid = (int)std::max<int64_t>(grid, std::min<int64_t>(resident, ceil_div(a.acc_words, kClearWordsPerCta)));
     if (R == 0) rounds = (int)ceil_div(a.M, (int64_t)kWarps * grid);  // kWarps rows per CTA and round
     // The grid barrier needs every CTA resident at once: a cooperative launch.
     cudaLaunchConfig_t cfg = {};
