@@ -5,7 +5,7 @@
 // Core of LLM.int8(): Mixed-precision Decomposition"; "Hugging Face LLM.int8()
 // integration" (agentlenshq.com), three-step recipe and CB/SCB weights.
 //
-// Kernels (HBM-bound streaming passes):
+// Kernels (the first four are HBM-bound streaming passes):
 //   prepare_weight_kernel  W [N,K] -> CB, SCB          (one warp per row)
 //   quantize_kernel        one cooperative launch: the CTA's rows of X are
 //                          staged in shared memory; phase A ORs the outlier
@@ -15,6 +15,12 @@
 //   quantize_stream_kernel prefill rows of 8192..16384 columns: X streamed
 //                          once, each row quantized with its own outliers
 //                          masked before the barrier and finished after it
+//   quantize_decode_kernel decode batches of up to 8 rows: one cluster owns
+//                          column slices of every row and exchanges the row
+//                          maxima and outlier counts through distributed
+//                          shared memory; no grid-wide step
+//   barrier_timeout_kernel a deliberately short-counted grid barrier that runs
+//                          out (failure-detection test of the bounded wait)
 //
 // Exactness: |x| >= threshold is decided on the fp16 bit pattern against the
 // smallest fp16 pattern whose value reaches the fp32 threshold (the map from
