@@ -1003,8 +1003,10 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
     grid_dep_launch();
     grid_dep_wait();
 
-    // Every CTA of the grid zeroes its share of the GEMV's partial sums.
-    {
+    // Every CTA of the grid zeroes its share of the GEMV's partial sums: the
+    // other clusters at once, the quantizing one after its passes, which are
+    // the critical path.
+    auto zero_share = [&]() {
         const int64_t b = (int64_t)blockIdx.x, nb = gridDim.x;
         const uint4 z = make_uint4(0, 0, 0, 0);
         if (a.acc) {
@@ -1017,8 +1019,11 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
             const int64_t n4 = a.cnt_words / 4, per = ceil_div(n4, nb);
             for (int64_t i = b * per + threadIdx.x; i < min(n4, (b + 1) * per); i += kThreads) cnt4[i] = z;
         }
+    };
+    if (!quantizer) {
+        zero_share();
+        return;
     }
-    if (!quantizer) return;
 
     // Pass 1: outlier columns of the slice (every row of X is here).
     for (int i = threadIdx.x; i < nw; i += kThreads) s_bits[i] = 0;
@@ -1131,6 +1136,7 @@ __global__ void __launch_bounds__(kThreads) quantize_decode_kernel(QuantizeArgs 
             ca2[v] = quant_vec8(x, sc);
         }
     }
+    zero_share();
     cluster_wait();
 }
 
