@@ -32,7 +32,8 @@ EXPORTS = [
     "int8lt_read_device_status", "int8lt_prepare_weight", "int8lt_quantize_rows",
     "int8lt_forward", "int8lt_forward_quantize", "int8lt_forward_matmul",
     "int8lt_forward_static_scratch", "int8lt_static_scratch_read_status",
-    "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_wait_timeout",
+    "int8lt_debug_gemm_i32", "int8lt_debug_gemm_schedule", "int8lt_debug_tile_order",
+    "int8lt_debug_wait_timeout",
     "int8lt_debug_barrier_timeout", "int8lt_debug_static_scratch_timeout", "int8lt_set_gemm_split",
     "int8lt_quantize_rows_zp", "int8lt_prepare_weight_zp", "int8lt_forward_zp",
     "int8lt_forward_zp_quantize", "int8lt_forward_zp_matmul",
@@ -69,6 +70,7 @@ _SIGS = {
     "int8lt_debug_barrier_timeout": (ctypes.c_int, [_P, _SZ, _I64, _P]),
     "int8lt_debug_static_scratch_timeout": (ctypes.c_int, [_I64, _P]),
     "int8lt_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_int]),
+    "int8lt_debug_tile_order": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P]),
     "int8lt_set_gemm_split": (ctypes.c_int, [ctypes.c_int]),
     "int8lt_quantize_rows_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "int8lt_prepare_weight_zp": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),

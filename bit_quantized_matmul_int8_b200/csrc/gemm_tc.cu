@@ -931,6 +931,18 @@ extern "C" int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int mod
     return n;
 }
 
+extern "C" int int8lt_debug_tile_order(int num_m, int num_n, int32_t *out) {
+    if (num_m < 1 || num_n < 1 || !out || (int64_t)num_m * num_n > (1 << 30)) return -1;
+    const int tiles = num_m * num_n;
+    for (int t = 0; t < tiles; ++t) {
+        int m, n;
+        int8lt::tile_mn(t, num_m, tiles, m, n);
+        out[2 * t] = m;
+        out[2 * t + 1] = n;
+    }
+    return tiles;
+}
+
 extern "C" int int8lt_set_gemm_split(int mode) {
     if (mode < 0 || mode > 2) return -1;
     return int8lt::g_split_mode.exchange(mode);

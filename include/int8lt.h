@@ -361,6 +361,17 @@ int int8lt_set_gemm_split(int mode);
 int int8lt_debug_gemm_schedule(int tiles, int nkb, int pairs, int mode, int32_t *out, int cap_rows);
 
 /*
+ * Test entry (host only, no GPU needed): the order in which the prefill GEMM
+ * visits its output tiles, for num_m tile rows (256 rows of Y each) and
+ * num_n tile columns (256 output channels each). Tile index t is the one the
+ * schedule above names; out[2t], out[2t + 1] receive its tile row and tile
+ * column (out holds 2 * num_m * num_n int32, caller-owned). Returns
+ * num_m * num_n, or -1 for bad arguments (a null out, a dimension below 1,
+ * more than 2^30 tiles).
+ */
+int int8lt_debug_tile_order(int num_m, int num_n, int32_t *out);
+
+/*
  * Test entry: launch one block that waits on a barrier nothing ever arrives
  * at, with the same bounded-wait routine the GEMM pipeline uses, limited to
  * `limit_ns` nanoseconds (1e3 .. 1e9). The kernel records INT8LT_ERR_TIMEOUT

@@ -1,4 +1,4 @@
-"""The prefill GEMM's tile schedule (data-parallel + stream-K), on the CPU.
+"""The prefill GEMM's tile schedule (data-parallel + stream-K) and tile order, on the CPU.
 
 int8lt_debug_gemm_schedule enumerates, on the host, the exact segments the
 kernel walks. Every (tile, k-block) must be computed exactly once; a split
@@ -104,3 +104,43 @@ def test_set_gemm_split_roundtrip(L):
             _lib.int8lt_set_gemm_split(7)
     finally:
         _lib.int8lt_set_gemm_split(prev)
+
+
+def tile_order(L, num_m, num_n):
+    out = np.full((num_m * num_n, 2), -1, np.int32)
+    assert L.int8lt_debug_tile_order(num_m, num_n, out.ctypes.data) == num_m * num_n
+    return out
+
+
+@pytest.mark.parametrize("num_m,num_n", [
+    (8, 16),     # 2048 x 4096: one group of 8 tile rows, the former order
+    (16, 64),    # 4096 x 16384
+    (32, 144),   # 8192 x 36864: four groups
+    (17, 3),     # a last group of one tile row
+    (13, 5), (1, 1), (1, 7), (9, 1), (24, 2),
+])
+def test_tile_order_is_a_grouped_permutation(L, num_m, num_n):
+    """Every output tile is visited once; tiles go in groups of 8 tile rows
+    (the last group may be shorter), tile column by tile column inside a group,
+    tile row fastest; a group is finished before the next one starts."""
+    o = tile_order(L, num_m, num_n)
+    seen = np.zeros((num_m, num_n), np.int32)
+    for m, n in o:
+        assert 0 <= m < num_m and 0 <= n < num_n
+        seen[m, n] += 1
+    assert (seen == 1).all()
+    t = 0
+    for g0 in range(0, num_m, 8):
+        rows = min(8, num_m - g0)
+        for n in range(num_n):
+            for m in range(g0, g0 + rows):
+                assert tuple(o[t]) == (m, n), (t, tuple(o[t]), (m, n))
+                t += 1
+    assert t == num_m * num_n
+
+
+def test_tile_order_bad_arguments(L):
+    out = np.zeros(2, np.int32)
+    assert L.int8lt_debug_tile_order(0, 1, out.ctypes.data) == -1
+    assert L.int8lt_debug_tile_order(1, 0, out.ctypes.data) == -1
+    assert L.int8lt_debug_tile_order(1, 1, None) == -1
